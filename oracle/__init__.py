@@ -1,0 +1,145 @@
+"""fp64 CPU oracle for exact attention (forward and backward).
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code with the
+CUDA library under ``exact_io_aware_60_b200/`` and imports nothing from it.
+
+The arithmetic lives in ``attn_oracle.c``: the plain definition of standard attention
+(score matrix materialised, textbook softmax, textbook chain rule), which FlashAttention
+reproduces exactly up to floating-point ordering (anthology note "NOTE-005:
+FlashAttention", Theorem 1; promptingindex page "FlashAttention: The IO-Aware Algorithm
+That Rewrote GPU Training Speed Records", section "Tiling").  This module only marshals
+numpy arrays into it.
+
+Pins: every function here is pinned by ``tests/test_oracle_pins.py`` (brute-force
+softmax without max shift, closed forms, invariants, central finite differences).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` into ``liboracle.so`` (gcc, OpenMP, portable -O3)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O3", "-fPIC", "-shared", "-fopenmp", "-std=c11", "-Wall",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            dp = ctypes.POINTER(ctypes.c_double)
+            lp = ctypes.POINTER(ctypes.c_long)
+            lib.oracle_attention_rows.restype = ctypes.c_int
+            lib.oracle_attention_rows.argtypes = [
+                dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_double, ctypes.c_int,
+                ctypes.c_long, lp, ctypes.c_long, dp, dp, dp, dp, dp]
+            lib.oracle_threads.restype = ctypes.c_int
+            lib.oracle_threads.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def threads() -> int:
+    """OpenMP threads the oracle uses."""
+    return int(_load().oracle_threads())
+
+
+def _f64(a):
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return a
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows=None,
+                   want_dkdv=True):
+    """Exact attention of one (batch, head) for the query rows ``rows``.
+
+    q, k, v, dout: ``[N, d]`` arrays (cast to fp64).  ``kv_len``: valid keys (None = N).
+    Returns a dict with ``o [R,d]``, ``lse [R]`` and, when ``dout`` is given, ``dq [R,d]``
+    and (if ``want_dkdv``) ``dk``, ``dv [N,d]`` summed over the given rows only.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    assert k.shape == (N, d) and v.shape == (N, d)
+    L = N if kv_len is None else int(kv_len)
+    if rows is None:
+        rows = np.arange(N, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+    o = np.zeros((R, d))
+    lse = np.zeros((R,))
+    dq = dk = dv = None
+    if dout is not None:
+        dout = _f64(dout)
+        assert dout.shape == (N, d)
+        dq = np.zeros((R, d))
+        if want_dkdv:
+            dk = np.zeros((N, d))
+            dv = np.zeros((N, d))
+    rc = _load().oracle_attention_rows(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), N, d, float(scale), int(bool(causal)), L,
+        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), R,
+        _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_rows failed with status {rc}")
+    out = {"o": o, "lse": lse}
+    if dout is not None:
+        out["dq"] = dq
+        if want_dkdv:
+            out["dk"] = dk
+            out["dv"] = dv
+    return out
+
+
+def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=None):
+    """Exact attention over ``[B, H, N, d]`` arrays, one (b, h) at a time.
+
+    ``kv_len``: per-batch valid key counts (length B) or None.  ``heads``: optional list
+    of (b, h) pairs to evaluate; the others are left as NaN in the outputs.
+    Returns ``o``, ``lse`` and, with ``dout``, ``dq``, ``dk``, ``dv`` as fp64 arrays.
+    """
+    q = np.asarray(q)
+    B, H, N, d = q.shape
+    o = np.full((B, H, N, d), np.nan)
+    lse = np.full((B, H, N), np.nan)
+    res = {"o": o, "lse": lse}
+    if dout is not None:
+        for name in ("dq", "dk", "dv"):
+            res[name] = np.full((B, H, N, d), np.nan)
+    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    for b, h in pairs:
+        L = None if kv_len is None else int(kv_len[b])
+        r = attention_rows(q[b, h], k[b, h], v[b, h], None if dout is None else dout[b, h],
+                           scale=scale, causal=causal, kv_len=L)
+        o[b, h] = r["o"]
+        lse[b, h] = r["lse"]
+        if dout is not None:
+            res["dq"][b, h] = r["dq"]
+            res["dk"][b, h] = r["dk"]
+            res["dv"][b, h] = r["dv"]
+    return res
