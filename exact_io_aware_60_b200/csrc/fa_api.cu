@@ -1,0 +1,246 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, TMA descriptor
+// encoding, grid selection and kernel launches.  All kernels live in this single
+// translation unit (they are included below), so the device status word needs no
+// relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+thread_local char t_last_error[256] = "";
+
+void record_cuda_error(cudaError_t e, const char *where) {
+    snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
+             (int)e);
+}
+
+// ---------------------------------------------------------------- device checks
+
+std::atomic<int> g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
+
+int check_device(int *dev_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaGetDevice");
+        return FA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    int st = g_dev_ok[dev].load(std::memory_order_relaxed);
+    if (st == 0) {
+        int major = 0, minor = 0;
+        e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e != cudaSuccess) {
+            record_cuda_error(e, "cudaDeviceGetAttribute");
+            return FA_ERR_CUDA;
+        }
+        st = (major == 10 && minor == 0) ? 1 : 2;
+        g_dev_ok[dev].store(st, std::memory_order_relaxed);
+    }
+    *dev_out = dev;
+    return st == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D view [BH][rows][cols] of a contiguous tensor; box = box_cols x box_rows x 1.
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes,
+              long long cols, long long rows, long long bh, int box_cols, int box_rows,
+              CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)bh};
+    cuuint64_t strides[2] = {(cuuint64_t)(cols * elem_bytes), (cuuint64_t)(cols * rows * elem_bytes)};
+    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return false;
+    }
+    return true;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int d, float scale, int dtype) {
+    if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    const long long bh = (long long)B * H;
+    if (bh >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    if (bh * (long long)N * d > FA_MAX_ELEMENTS) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+template <typename K>
+cudaError_t set_smem(K kern, int bytes, std::atomic<int> *done, int dev) {
+    if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[dev].store(1, std::memory_order_relaxed);
+    return e;
+}
+
+template <int D, bool BF16>
+int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+               int N, float scale, int causal, const int *kv_len, cudaStream_t st, int dev) {
+    using C = fa::FwdCfg<D>;
+    const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const long long bh = (long long)B * H;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, q, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, k, dt, 2, D, N, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, v, dt, 2, D, N, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mo, o, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return FA_ERR_CUDA;
+    fa::FwdParams p;
+    p.lse = lse;
+    p.kv_len = kv_len;
+    p.N = N;
+    p.BH = (int)bh;
+    p.H = H;
+    p.num_q_tiles = (N + C::BM - 1) / C::BM;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    auto kern = fa::fa_fwd_kernel<D, BF16>;
+    static std::atomic<int> smem_done[kMaxDevices];
+    cudaError_t e = set_smem(kern, C::SMEM, smem_done, dev);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaFuncSetAttribute(fwd)");
+        return FA_ERR_CUDA;
+    }
+    const long long grid = (long long)p.num_q_tiles * bh;
+    if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "fa_fwd launch");
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return kVersion; }
+
+const char *fa_strerror(int status) {
+    switch (status) {
+        case FA_OK: return "ok";
+        case FA_ERR_INVALID_ARG: return "invalid argument";
+        case FA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case FA_ERR_CUDA: return "CUDA error";
+        case FA_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char *fa_last_cuda_error(void) { return t_last_error; }
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
+           int d, float scale, int causal, const int *kv_len, int dtype, void *stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, N, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    int dev = 0;
+    rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+    if (d == 64)
+        return bf16 ? launch_fwd<64, true>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev)
+                    : launch_fwd<64, false>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev);
+    return bf16 ? launch_fwd<128, true>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev)
+                : launch_fwd<128, false>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+    const size_t rows = (size_t)B * H * N;
+    const size_t dq = (rows * d * 4 + 255) & ~(size_t)255;
+    const size_t dd = (rows * 4 + 255) & ~(size_t)255;
+    return dq + dd;
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+           float scale, int causal, const int *kv_len, int dtype, void *workspace,
+           size_t workspace_bytes, void *stream) {
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
+        return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+    if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, N, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+    int dev = 0;
+    rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    (void)causal;
+    return FA_ERR_UNSUPPORTED;
+}
+
+int fa_get_device_status(void *stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaStreamSynchronize");
+        return FA_ERR_CUDA;
+    }
+    int val = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&val, fa::g_status, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "status word");
+        return FA_ERR_CUDA;
+    }
+    return val == 0 ? FA_OK : FA_ERR_TIMEOUT;
+}
+
+}  // extern "C"

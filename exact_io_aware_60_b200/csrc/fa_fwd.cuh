@@ -1,0 +1,342 @@
+// fa_fwd.cuh -- forward pass of exact tiled attention on sm_100a.
+//
+// The method (anthology note "NOTE-005: FlashAttention", section "Method"; aicassindra
+// FlashAttention architecture page, "End-to-end flow"): split Q into row blocks and
+// K, V into key blocks, bring one block at a time on chip, form that block of scores
+// there, and fold it into the output with an online softmax that carries a running row
+// maximum m and normaliser l, rescaling the accumulated output whenever m grows.  Only
+// O and the row statistics leave the chip; the N x N score matrix never exists in HBM.
+//
+// B200 mapping (one CTA = one 128-row query tile of one (batch, head)):
+//   warp 4      TMA producer: Q once, then K_j / V_j into an NS-stage shared-memory ring
+//               (128-byte swizzle, mbarrier transaction counts).
+//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM (double-buffered, so the
+//               next block's scores are computed while softmax works on this one), then
+//               O += P_j V_j with P_j read straight from TMEM.
+//   warps 0..3  softmax, one query row per thread (TMEM lane = row): load S_j, mask on
+//               diagonal / tail blocks only, row max, p = 2^(s*scale*log2e - m) with the
+//               MUFU ex2, row sum, P_j written back into TMEM as 16-bit pairs over S_j.
+//               The output rescale is lazy: m only moves when the row max grows by more
+//               than 2^8, which leaves the result exact because O and l always share the
+//               same m.  Epilogue: O / l -> 16-bit, staged swizzled in shared memory and
+//               written with one TMA store; LSE = ln2 * (m + log2 l).
+// The loop order is query-block outer (each CTA writes its O rows once) instead of the
+// key-block-outer order of the original algorithm; the result is the same up to
+// floating-point ordering.
+#pragma once
+
+#include <cuda.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+struct FwdParams {
+    float *lse;
+    const int *kv_len;
+    int N;
+    int BH;
+    int H;
+    int num_q_tiles;
+    float scale_log2;  // scale * log2(e)
+    int causal;
+};
+
+template <int D>
+struct FwdCfg {
+    static constexpr int BM = 128;                      // query rows per tile
+    static constexpr int BN = 128;                      // keys per block
+    static constexpr int HALVES = D / 64;               // 128-byte column blocks per row
+    static constexpr int TILE = BM * D * 2;             // bytes of one Q / K / V tile
+    static constexpr int HALF = BM * 128;               // bytes of one column block
+    static constexpr int NS = (D == 64) ? 4 : 2;        // K/V ring depth
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + TILE;
+    static constexpr int OFF_V = OFF_K + NS * TILE;
+    static constexpr int OFF_BAR = OFF_V + NS * TILE;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;   // + barriers + alignment slack
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_O = 256;              // S0 at 0, S1 at 128, O at 256
+};
+
+struct FwdBars {
+    uint64_t q_full;
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_full;
+    uint64_t k_full[4];
+    uint64_t v_full[4];
+    uint64_t kv_empty[4];
+    uint32_t tmem_base;
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(192, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    uint8_t *sQ = smem + C::OFF_Q;
+    uint8_t *sK = smem + C::OFF_K;
+    uint8_t *sV = smem + C::OFF_V;
+    FwdBars *bars = reinterpret_cast<FwdBars *>(smem + C::OFF_BAR);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: heaviest causal tiles are launched first.
+    const int tile_rank = blockIdx.x / p.BH;
+    const int bh = blockIdx.x - tile_rank * p.BH;
+    const int qt = p.causal ? (p.num_q_tiles - 1 - tile_rank) : tile_rank;
+    const int b = bh / p.H;
+    int L = p.N;
+    if (p.kv_len != nullptr) {
+        L = p.kv_len[b];
+        L = L < 0 ? 0 : (L > p.N ? p.N : L);
+    }
+    int kv_end = L;
+    if (p.causal) kv_end = min(kv_end, (qt + 1) * C::BM);
+    const int T = (kv_end + C::BN - 1) / C::BN;  // key blocks this tile visits
+
+    if (threadIdx.x == 128) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
+        mbar_init(&bars->q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 128);
+        }
+        mbar_init(&bars->o_full, 1);
+        for (int i = 0; i < C::NS; ++i) {
+            mbar_init(&bars->k_full[i], 1);
+            mbar_init(&bars->v_full[i], 1);
+            mbar_init(&bars->kv_empty[i], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 5) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0 && T > 0) {
+            mbar_arrive_expect_tx(&bars->q_full, C::TILE);
+            for (int hf = 0; hf < C::HALVES; ++hf)
+                tma_load_3d(sQ + hf * C::HALF, &tmQ, &bars->q_full, hf * 64, qt * C::BM, bh);
+            for (int j = 0; j < T; ++j) {
+                const int s = j % C::NS;
+                if (j >= C::NS && !mbar_wait(&bars->kv_empty[s], ((j / C::NS) - 1) & 1)) break;
+                mbar_arrive_expect_tx(&bars->k_full[s], C::TILE);
+                for (int hf = 0; hf < C::HALVES; ++hf)
+                    tma_load_3d(sK + s * C::TILE + hf * C::HALF, &tmK, &bars->k_full[s], hf * 64,
+                                j * C::BN, bh);
+                mbar_arrive_expect_tx(&bars->v_full[s], C::TILE);
+                for (int hf = 0; hf < C::HALVES; ++hf)
+                    tma_load_3d(sV + s * C::TILE + hf * C::HALF, &tmV, &bars->v_full[s], hf * 64,
+                                j * C::BN, bh);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0 && T > 0) {
+            constexpr uint32_t kIdescS = idesc_f16(BF16, false, false, 128, 128);
+            constexpr uint32_t kIdescO = idesc_f16(BF16, false, true, 128, D);
+            const uint32_t q_addr = smem_u32(sQ);
+            const uint32_t k_addr = smem_u32(sK);
+            const uint32_t v_addr = smem_u32(sV);
+            bool ok = mbar_wait(&bars->q_full, 0);
+            tc_fence_after();
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % C::NS;
+                if (!mbar_wait(&bars->k_full[s], (j / C::NS) & 1)) return false;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 128);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * C::HALF + (kk & 3) * 32);
+                    const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(k_addr + s * C::TILE + off, 16, 1024);
+                    mma_ss(d_tmem, a, bd, kIdescS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars->s_full[j & 1]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < T; ++j) {
+                if (j + 1 < T && !issue_s(j + 1)) break;
+                const int s = j % C::NS;
+                if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1)) break;
+                if (!mbar_wait(&bars->v_full[s], (j / C::NS) & 1)) break;
+                tc_fence_after();
+                const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 128);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint64_t bd =
+                        smem_desc_sw128(v_addr + s * C::TILE + kk * 2048, C::HALF, 1024);
+                    mma_ts(tmem + C::COL_O, p_tmem + kk * 8, bd, kIdescO,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&bars->kv_empty[s]);
+                mma_commit(&bars->o_full);
+            }
+        }
+    } else {
+        // ------------------------------ softmax warps ------------------------------
+        const int t = threadIdx.x;  // 0..127: row in the tile and TMEM lane
+        const int row = qt * C::BM + t;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        float m = -INFINITY;  // running max, in units of log2 (already scaled)
+        float l = 0.f;        // running normaliser
+        bool ok = true;
+        for (int j = 0; j < T; ++j) {
+            if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sb = tmem + lane_base + (uint32_t)((j & 1) * 128);
+            float s[128];
+            {
+                uint32_t r[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    tmem_ld32(sb + c * 32, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                }
+            }
+            const bool need_mask = ((j + 1) * C::BN > L) || (p.causal && j == qt);
+            if (need_mask) {
+                const int lim = p.causal ? min(L, row + 1) : L;  // keys < lim are visible
+                const int c0 = lim - j * C::BN;
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= c0) s[c] = -INFINITY;
+            }
+            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+            for (int c = 4; c < 128; c += 4) {
+                mx0 = fmaxf(mx0, s[c]);
+                mx1 = fmaxf(mx1, s[c + 1]);
+                mx2 = fmaxf(mx2, s[c + 2]);
+                mx3 = fmaxf(mx3, s[c + 3]);
+            }
+            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            // Lazy rescale: move m only when the max grew by more than 2^8.
+            const bool grow = mx > m + 8.0f;
+            const bool any_grow = __any_sync(0xffffffffu, grow);
+            float alpha = 1.f;
+            if (any_grow && mx > m) {
+                alpha = ex2(m - mx);  // m == -inf gives 0
+                m = mx;
+            }
+            const float m_use = (m == -INFINITY) ? 0.f : m;
+            float sum0 = 0.f, sum1 = 0.f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < 128; c += 2) {
+                const float p0 = ex2(fmaf(s[c], sl2, -m_use));
+                const float p1 = ex2(fmaf(s[c + 1], sl2, -m_use));
+                sum0 += p0;
+                sum1 += p1;
+                pk[c >> 1] = pack2<BF16>(p0, p1);
+            }
+            l = l * alpha + (sum0 + sum1);
+            {
+                uint32_t r[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = pk[i];
+                tmem_st32(sb, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = pk[32 + i];
+                tmem_st32(sb + 32, r);
+            }
+            // Every phase of o_full is waited on, in order, so that a parity wait can
+            // never alias a phase two ahead.  P_{j-1} V_{j-1} was issued a whole softmax
+            // block ago, so this wait is normally already satisfied.
+            if (j > 0) {
+                if (!mbar_wait(&bars->o_full, (j - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+            }
+            if (j > 0 && any_grow) {
+                // Rescale the accumulated output (P_{j-1} V_{j-1} is complete).
+                const uint32_t ob = tmem + lane_base + C::COL_O;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(ob + c * 32, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(ob + c * 32, r);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[j & 1]);
+        }
+
+        // ------------------------------ epilogue ------------------------------
+        if (ok && T > 0) {
+            ok = mbar_wait(&bars->o_full, (T - 1) & 1);
+            tc_fence_after();
+        }
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        const uint32_t ob = tmem + lane_base + C::COL_O;
+#pragma unroll
+        for (int hf = 0; hf < C::HALVES; ++hf) {
+            uint32_t w[32];
+            {
+                uint32_t r[32];
+                if (T > 0) {
+                    tmem_ld32(ob + hf * 64, r);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv,
+                                       __uint_as_float(r[2 * i + 1]) * inv);
+                if (T > 0) {
+                    tmem_ld32(ob + hf * 64 + 32, r);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[16 + i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv,
+                                            __uint_as_float(r[2 * i + 1]) * inv);
+            }
+            // Row t of this 128-byte column block, 16-byte chunks XOR-swizzled by t % 8.
+            uint8_t *rowp = sQ + hf * C::HALF + t * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 v4 = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                *reinterpret_cast<uint4 *>(rowp + ((c ^ (t & 7)) << 4)) = v4;
+            }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (t == 0) {
+            for (int hf = 0; hf < C::HALVES; ++hf)
+                tma_store_3d(&tmO, sQ + hf * C::HALF, hf * 64, qt * C::BM, bh);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();
+        }
+        if (row < p.N) {
+            const float lse = (l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
+            p.lse[(size_t)bh * p.N + row] = lse;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace fa

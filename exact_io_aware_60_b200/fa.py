@@ -1,0 +1,186 @@
+"""ctypes binding of libfa.so (declared in include/fa.h).
+
+The functions named like the C entry points (``fa_fwd``, ``fa_bwd``, ...) only marshal
+arguments: they check shapes and dtypes, take raw device pointers from torch tensors
+and pass the current CUDA stream.  Every step of the computation runs in the library's
+CUDA kernels.  ``forward`` / ``backward`` additionally allocate the outputs with torch.
+
+The library is loaded on first use.  If ``libfa.so`` is missing, or a call returns an
+error, a :class:`FAError` is raised: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_BF16, FA_FP16 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        detail = ""
+        if _lib is not None:
+            detail = _lib.fa_last_cuda_error().decode()
+        msg = f"{where}: {fa_strerror(status)} (status {status})"
+        if status == FA_ERR_CUDA and detail:
+            msg += f": {detail}"
+        super().__init__(msg)
+
+
+def lib():
+    """The loaded ctypes library (raises if libfa.so has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise FAError(FA_ERR_UNSUPPORTED,
+                              f"libfa.so not found at {LIB_PATH} (build it with "
+                              "`python -m exact_io_aware_60_b200.build`)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            L.fa_fwd.restype = i
+            L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, i, vp]
+            L.fa_bwd.restype = i
+            L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, i,
+                                 vp, sz, vp]
+            L.fa_bwd_workspace_bytes.restype = sz
+            L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+            L.fa_strerror.restype = ctypes.c_char_p
+            L.fa_strerror.argtypes = [i]
+            L.fa_last_cuda_error.restype = ctypes.c_char_p
+            L.fa_last_cuda_error.argtypes = []
+            L.fa_get_device_status.restype = i
+            L.fa_get_device_status.argtypes = [vp]
+            L.fa_version.restype = i
+            L.fa_version.argtypes = []
+            _lib = L
+    return _lib
+
+
+def fa_strerror(status: int) -> str:
+    if _lib is None:
+        return {0: "ok", 1: "invalid argument", 2: "unsupported configuration or device",
+                3: "CUDA error", 4: "device-side wait timed out"}.get(status, "unknown status")
+    return _lib.fa_strerror(int(status)).decode()
+
+
+def fa_version() -> int:
+    return int(lib().fa_version())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise FAError(FA_ERR_INVALID_ARG, f"unsupported dtype {t.dtype}")
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype):
+    if not isinstance(t, torch.Tensor):
+        raise FAError(FA_ERR_INVALID_ARG, f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise FAError(FA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise FAError(FA_ERR_INVALID_ARG,
+                      f"{name}: expected contiguous {dtype} {tuple(shape)}, got "
+                      f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()}")
+
+
+def _kv_ptr(kv_len, B):
+    if kv_len is None:
+        return None
+    _check(kv_len, "kv_len", (B,), torch.int32)
+    return kv_len.data_ptr()
+
+
+def fa_fwd(q, k, v, o, lse, *, scale: float, causal: bool = False, kv_len=None,
+           stream=None) -> None:
+    """Enqueues the forward pass: writes ``o`` ([B,H,N,d]) and ``lse`` ([B,H,N] fp32)."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, float(scale), int(bool(causal)), _kv_ptr(kv_len, B),
+                      _dtype_code(q), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd")
+
+
+def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: bool = False,
+           kv_len=None, workspace: torch.Tensor, stream=None) -> None:
+    """Enqueues the backward pass: writes ``dq``, ``dk``, ``dv``.  ``workspace`` is a
+    uint8 CUDA tensor of at least ``fa_bwd_workspace_bytes`` bytes."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise FAError(FA_ERR_INVALID_ARG, "workspace must be a contiguous uint8 CUDA tensor")
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                      float(scale), int(bool(causal)), _kv_ptr(kv_len, B), _dtype_code(q),
+                      workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd")
+
+
+def fa_get_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status word."""
+    return int(lib().fa_get_device_status(_stream_handle(stream)))
+
+
+# ------------------------------------------------------------------ conveniences
+
+def forward(q, k, v, *, scale: Optional[float] = None, causal: bool = False, kv_len=None,
+            stream=None):
+    """Allocates ``o`` and ``lse`` with torch and runs :func:`fa_fwd`."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, scale=scale, causal=causal, kv_len=kv_len, stream=stream)
+    return o, lse
+
+
+def workspace_for(q) -> torch.Tensor:
+    B, H, N, d = q.shape
+    return torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+
+
+def backward(q, k, v, o, dout, lse, *, scale: Optional[float] = None, causal: bool = False,
+             kv_len=None, workspace=None, stream=None):
+    """Allocates ``dq``, ``dk``, ``dv`` (and the workspace if not given) and runs
+    :func:`fa_bwd`."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = workspace_for(q)
+    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scale=scale, causal=causal, kv_len=kv_len,
+           workspace=workspace, stream=stream)
+    return dq, dk, dv

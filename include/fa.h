@@ -1,0 +1,137 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa.so).
+ *
+ * The library computes exact attention O = softmax(scale * Q K^T + mask) V and its
+ * gradients without ever forming the N x N score matrix in device memory:
+ *   - the method: tile Q, K, V into on-chip blocks and update the output with an
+ *     online softmax that carries a running row maximum m and normaliser l
+ *     (anthology note "NOTE-005: FlashAttention", section "Method"; aicassindra
+ *     FlashAttention architecture page, "End-to-end flow");
+ *   - exactness: the result equals standard attention up to floating-point ordering
+ *     (NOTE-005, Theorem 1; promptingindex page "FlashAttention: The IO-Aware
+ *     Algorithm That Rewrote GPU Training Speed Records", section "Tiling");
+ *   - the backward pass recomputes each probability block from the stored
+ *     statistics instead of reading a saved matrix (NOTE-005, "Method" and "Key
+ *     components"; aicassindra page, "The architecture: every piece explained").
+ * The forward pass stores the two statistics as one array, the log-sum-exp
+ * LSE_i = m_i + ln l_i (natural log).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous row-major [B, H, N, d] arrays of
+ *   the element type `dtype` (d innermost).  LSE is a contiguous fp32 [B, H, N] array.
+ *   Q, K and V share the sequence length N (self-attention).
+ * Mask: key j is visible to query i iff j < L_b and (causal == 0 or j <= i), with
+ *   L_b = kv_len[b] clamped to [0, N], or L_b = N when kv_len is NULL.  kv_len, when
+ *   given, is a DEVICE pointer to B int32 values.  Masked scores are -inf.  A query
+ *   row that sees no key (only when L_b = 0) gets O = 0, LSE = -inf and zero gradient.
+ * Scale: `scale` multiplies Q K^T before masking; it must be finite and > 0
+ *   (typically 1/sqrt(d)).
+ * Supported: d in {64, 128}; dtype FA_BF16 or FA_FP16 (fp32 accumulation inside);
+ *   any N >= 1, B >= 1, H >= 1, B*H < 2^31, and at most FA_MAX_ELEMENTS elements in
+ *   one [B, H, N, d] tensor.  Device: compute capability 10.0 (B200, sm_100a) only.
+ * Pointers: all tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
+ *   caller; the library never allocates, frees or retains them after the call.
+ * Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  Every entry
+ *   point only enqueues work on `stream` and returns; results are ready once the
+ *   stream is synchronised.
+ * Errors: arguments are checked before anything is enqueued.  FA_ERR_INVALID_ARG:
+ *   null or misaligned pointer, non-positive size, bad scale or dtype, workspace
+ *   too small.  FA_ERR_UNSUPPORTED: d not 64/128, tensor too large, device not
+ *   sm_100.  FA_ERR_CUDA: a CUDA call or launch failed (see fa_last_cuda_error()).
+ *   There is no fallback of any kind: an unsupported call does no work.
+ * Device-side waits are bounded.  A wait that gives up records FA_ERR_TIMEOUT in a
+ *   per-device status word readable with fa_get_device_status().
+ * Thread safety: every entry point may be called concurrently from several host
+ *   threads; the only global state is a per-device status word and cached device
+ *   properties.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,
+    FA_ERR_UNSUPPORTED = 2,
+    FA_ERR_CUDA = 3,
+    FA_ERR_TIMEOUT = 4
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/* Largest element count of one [B, H, N, d] tensor the kernels index. */
+#define FA_MAX_ELEMENTS ((long long)1 << 40)
+
+/*
+ * Forward pass (NOTE-005 "Method": tiles of Q against all K/V tiles, online softmax
+ * with running m and l; output O and the row statistics).
+ *   q, k, v : [B, H, N, d] dtype, read only.
+ *   o       : [B, H, N, d] dtype, written.
+ *   lse     : [B, H, N] fp32, written; LSE_i = ln sum_j exp(scale q_i.k_j) over the
+ *             visible keys (-inf for a row that sees none).
+ *   kv_len  : NULL or device int32[B] (see Mask above).
+ * Returns FA_OK or an error code (nothing is enqueued on error).
+ */
+FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int H, int N, int d, float scale, int causal, const int *kv_len,
+           int dtype, void *stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes: an fp32 [B, H, N, d] dQ
+ * accumulator and an fp32 [B, H, N] array D_i = sum_c dO_ic O_ic, each 256-byte
+ * aligned.  Returns 0 for invalid sizes.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass of the loss sum(O * dO): recomputes every probability block from
+ * q, k and the stored lse (NOTE-005 "Method": recompute rather than read a saved
+ * matrix) and writes dQ, dK, dV.
+ *   q, k, v, o, dout : [B, H, N, d] dtype, read only (o and lse from fa_fwd with the
+ *                      same q, k, v, scale, causal and kv_len).
+ *   lse              : [B, H, N] fp32, read only.
+ *   dq, dk, dv       : [B, H, N, d] dtype, written (rows of dK/dV for keys >= L_b
+ *                      are written as exact zeros).
+ *   workspace        : device buffer of at least fa_bwd_workspace_bytes() bytes,
+ *                      256-byte aligned; its contents on entry do not matter and
+ *                      are clobbered.
+ * Enqueues three kernels on `stream` (row-dot preprocess, main pass, dQ convert).
+ */
+FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+           float scale, int causal, const int *kv_len, int dtype, void *workspace,
+           size_t workspace_bytes, void *stream);
+
+/* Static, NUL-terminated description of a status code. */
+FA_API const char *fa_strerror(int status);
+
+/* Text of the last CUDA error this host thread saw inside the library ("" if none). */
+FA_API const char *fa_last_cuda_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status word.
+ * Returns FA_OK, FA_ERR_TIMEOUT if some kernel gave up a bounded wait since the
+ * last call, or FA_ERR_CUDA if the synchronisation failed.
+ */
+FA_API int fa_get_device_status(void *stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

@@ -1,0 +1,104 @@
+"""The C-ABI library loads, exports every entry point include/fa.h declares, and its
+host-side argument checks reject bad calls before touching CUDA (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_60_b200 import fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"^FA_API\s+[\w\s\*]*?\b(fa_\w+)\s*\(", src, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_strerror",
+              "fa_get_device_status", "fa_last_cuda_error", "fa_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_version_and_strerror():
+    assert fa.fa_version() >= 100
+    L = fa.lib()
+    for code in range(5):
+        assert L.fa_strerror(code).decode() == fa.fa_strerror(code)
+    assert L.fa_strerror(99).decode() == "unknown status"
+
+
+def test_workspace_bytes():
+    L = fa.lib()
+    n = L.fa_bwd_workspace_bytes(2, 3, 100, 64)
+    rows = 2 * 3 * 100
+    assert n == ((rows * 64 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    assert L.fa_bwd_workspace_bytes(0, 3, 100, 64) == 0
+
+
+GOOD = dict(B=1, H=1, N=16, d=64, scale=0.125, causal=0, dtype=0)
+P = 4096  # fake, 16-byte aligned non-null "device" address: never dereferenced
+
+
+def call_fwd(**over):
+    a = dict(GOOD, q=P, k=P, v=P, o=P, lse=P, kv=None)
+    a.update(over)
+    return fa.lib().fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"],
+                           a["d"], a["scale"], a["causal"], a["kv"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=None), fa.FA_ERR_INVALID_ARG),
+    (dict(k=P + 8), fa.FA_ERR_INVALID_ARG),
+    (dict(kv=P + 2), fa.FA_ERR_INVALID_ARG),
+    (dict(B=0), fa.FA_ERR_INVALID_ARG),
+    (dict(N=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(dtype=7), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(B=1 << 16, H=1 << 15), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_bad_arguments_on_host(over, code):
+    assert call_fwd(**over) == code
+
+
+def call_bwd(**over):
+    a = dict(GOOD, ptr=P, ws=P * 16, wsb=1 << 30, kv=None)
+    a.update(over)
+    p = a["ptr"]
+    return fa.lib().fa_bwd(p, p, p, p, p, p, p, p, p, a["B"], a["H"], a["N"], a["d"],
+                           a["scale"], a["causal"], a["kv"], a["dtype"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(ptr=None), fa.FA_ERR_INVALID_ARG),
+    (dict(ptr=P + 4), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=None), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=P * 16 + 16), fa.FA_ERR_INVALID_ARG),
+    (dict(wsb=16), fa.FA_ERR_INVALID_ARG),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+])
+def test_bwd_rejects_bad_arguments_on_host(over, code):
+    assert call_bwd(**over) == code
+
+
+def test_binding_raises_without_cuda_tensors():
+    import torch
+    x = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(fa.FAError):
+        fa.fa_fwd(x, x, x, x, torch.zeros(1, 1, 4), scale=0.1)
