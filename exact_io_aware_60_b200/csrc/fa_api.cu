@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -158,6 +159,120 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     return FA_OK;
 }
 
+
+struct BwdWorkspace {
+    float *dq_acc;
+    float *lse2;
+    float *dvec;
+    size_t total;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+BwdWorkspace bwd_workspace_layout(void *base, long long BH, int N, int d) {
+    const int npad = ((N + 127) / 128) * 128;
+    const size_t dq = round256((size_t)BH * N * d * 4);
+    const size_t vec = round256((size_t)BH * npad * 4);
+    BwdWorkspace w;
+    char *b = static_cast<char *>(base);
+    w.dq_acc = reinterpret_cast<float *>(b);
+    w.lse2 = reinterpret_cast<float *>(b + dq);
+    w.dvec = reinterpret_cast<float *>(b + dq + vec);
+    w.total = dq + 2 * vec;
+    return w;
+}
+
+int grid_for(long long work, int threads) {
+    long long g = (work + threads - 1) / threads;
+    if (g < 1) g = 1;
+    if (g > 148LL * 16) g = 148LL * 16;
+    return (int)g;
+}
+
+template <int D, bool BF16>
+int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+               const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, float scale,
+               int causal, const int *kv_len, void *workspace, cudaStream_t st, int dev) {
+    using C = fa::BwdCfg<D>;
+    const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const long long bh = (long long)B * H;
+    const int num_tiles = (N + 127) / 128;
+    BwdWorkspace ws = bwd_workspace_layout(workspace, bh, N, D);
+
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
+    if (!make_map(&mq, q, dt, 2, D, N, bh, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, k, dt, 2, D, N, bh, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, v, dt, 2, D, N, bh, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mdo, dout, dt, 2, D, N, bh, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mdk, dk, dt, 2, D, N, bh, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mdv, dv, dt, 2, D, N, bh, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mdq, ws.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, bh, 32, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return FA_ERR_CUDA;
+
+    // 1. D = rowsum(dO o O), LSE in base 2, zeroed dQ accumulator.
+    fa::BwdPrepParams pp;
+    pp.o = o;
+    pp.dout = dout;
+    pp.lse = lse;
+    pp.lse2 = ws.lse2;
+    pp.dvec = ws.dvec;
+    pp.dq_acc = reinterpret_cast<float4 *>(ws.dq_acc);
+    pp.dq_acc_vec4 = bh * (long long)N * D / 4;
+    pp.N = N;
+    pp.Npad = num_tiles * 128;
+    pp.BH = bh;
+    const long long prep_work = std::max(pp.dq_acc_vec4, bh * pp.Npad * (D / 8));
+    fa::fa_bwd_prep_kernel<D, BF16><<<grid_for(prep_work, 256), 256, 0, st>>>(pp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "fa_bwd prep launch");
+        return FA_ERR_CUDA;
+    }
+
+    // 2. main pass
+    fa::BwdParams p;
+    p.lse2 = ws.lse2;
+    p.dvec = ws.dvec;
+    p.dq_acc = ws.dq_acc;
+    p.kv_len = kv_len;
+    p.N = N;
+    p.Npad = num_tiles * 128;
+    p.BH = (int)bh;
+    p.H = H;
+    p.num_tiles = num_tiles;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    auto kern = fa::fa_bwd_kernel<D, BF16>;
+    static std::atomic<int> smem_done[kMaxDevices];
+    e = set_smem(kern, C::SMEM, smem_done, dev);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaFuncSetAttribute(bwd)");
+        return FA_ERR_CUDA;
+    }
+    const long long grid = (long long)num_tiles * bh;
+    if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "fa_bwd launch");
+        return FA_ERR_CUDA;
+    }
+
+    // 3. dQ = scale * dQ_acc in the input dtype
+    const long long nv4 = bh * (long long)N * D / 4;
+    fa::fa_bwd_convert_kernel<BF16><<<grid_for(nv4, 256), 256, 0, st>>>(
+        reinterpret_cast<const float4 *>(ws.dq_acc), reinterpret_cast<uint2 *>(dq), nv4, scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "fa_bwd convert launch");
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -199,10 +314,7 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
     if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
-    const size_t rows = (size_t)B * H * N;
-    const size_t dq = (rows * d * 4 + 255) & ~(size_t)255;
-    const size_t dd = (rows * 4 + 255) & ~(size_t)255;
-    return dq + dd;
+    return bwd_workspace_layout(nullptr, (long long)B * H, N, d).total;
 }
 
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
@@ -222,8 +334,13 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
     int dev = 0;
     rc = check_device(&dev);
     if (rc != FA_OK) return rc;
-    (void)causal;
-    return FA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, workspace, st, dev
+    if (d == 64)
+        return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
+    return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
+#undef FA_BWD_ARGS
 }
 
 int fa_get_device_status(void *stream) {

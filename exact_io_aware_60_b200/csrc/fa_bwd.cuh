@@ -1,3 +1,547 @@
-// fa_bwd.cuh -- backward pass (to be filled in).
+// fa_bwd.cuh -- backward pass of exact tiled attention on sm_100a.
+//
+// The method (anthology note "NOTE-005: FlashAttention", sections "Method" and "Key
+// components"; aicassindra FlashAttention architecture page, "The architecture: every
+// piece explained"): the backward pass does not read a stored N x N probability matrix;
+// it recomputes each probability block on chip from Q, K and the statistics the forward
+// pass kept (here LSE = m + ln l), then applies the chain rule of the op chain
+//   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P o (dP - D),
+//   dQ = scale dS K,  dK = scale dS^T Q.
+// (The pages state the recomputation but print no gradient formulas; these are the
+// textbook derivatives of softmax and of the two products.)
+//
+// Three kernels, all on the caller's stream:
+//   1. fa_bwd_prep_kernel: D_i = rowsum(dO o O) in fp32, LSE in base 2 (padded to whole
+//      128-row tiles, +inf where there is no row), and zeroes the fp32 dQ accumulator.
+//   2. fa_bwd_kernel: one CTA per 128-key tile of one (batch, head), looping over the
+//      128-query tiles that can see it (causal: only tiles on or below the diagonal).
+//        warp 4      TMA producer: K, V once; Q_i, dO_i (+ LSE_i, D_i) into a 2-stage ring.
+//        warp 5      MMA issuer (one thread), all on tcgen05 with fp32 TMEM accumulators:
+//                    S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i, dK += dS^T Q_i
+//                    (P^T, dS^T read from TMEM), dQ_i = dS K (dS from shared memory).
+//        warps 0..3  one key row per thread: P^T = 2^(S^T scale log2e - LSE2), written back
+//                    to TMEM as 16-bit pairs; dS^T = P^T o (dP^T - D) to TMEM and, in the
+//                    transposed operand layout, to shared memory; epilogue writes dK, dV.
+//        warps 6..9  drain dQ_i from TMEM and add it into the fp32 accumulator in global
+//                    memory (TMA reduce-add of a swizzled staging tile for d = 64; vector
+//                    red.global.add for d = 128, where shared memory is fully used).
+//   3. fa_bwd_convert_kernel: dQ = scale * dQ_acc in the input dtype.
 #pragma once
+
+#include <cuda.h>
+
 #include "sm100.cuh"
+
+namespace fa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// --------------------------------------------------------------------------- prep
+
+struct BwdPrepParams {
+    const void *o;
+    const void *dout;
+    const float *lse;
+    float *lse2;   // [BH][Npad]
+    float *dvec;   // [BH][Npad]
+    float4 *dq_acc;
+    long long dq_acc_vec4;  // number of float4 in dq_acc
+    int N;
+    int Npad;
+    long long BH;
+};
+
+// Each warp handles 32 / (D/8) consecutive padded rows per step (D/8 threads per row,
+// 8 elements of O and dO each); every lane runs the same number of steps, so the
+// group shuffles never diverge.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p) {
+    constexpr int G = D / 8;           // threads per row
+    constexpr int RPW = 32 / G;        // rows per warp step
+    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long nthreads = (long long)gridDim.x * blockDim.x;
+    for (long long i = tid; i < p.dq_acc_vec4; i += nthreads)
+        p.dq_acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const long long rows_total = p.BH * p.Npad;
+    const int lane = threadIdx.x & 31;
+    const int g = lane % G;
+    const long long warp_id = tid >> 5;
+    const long long nwarps = nthreads >> 5;
+    for (long long base = warp_id * RPW; base < rows_total; base += nwarps * RPW) {
+        const long long rr = base + lane / G;
+        float acc = 0.f;
+        float l2 = INFINITY;
+        if (rr < rows_total) {
+            const long long bh = rr / p.Npad;
+            const int r = (int)(rr - bh * p.Npad);
+            if (r < p.N) {
+                const size_t off = ((size_t)bh * p.N + r) * D + g * 8;
+                const uint4 a = *reinterpret_cast<const uint4 *>(
+                    reinterpret_cast<const uint16_t *>(p.o) + off);
+                const uint4 bb = *reinterpret_cast<const uint4 *>(
+                    reinterpret_cast<const uint16_t *>(p.dout) + off);
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 x = unpack2<BF16>(aw[k]);
+                    const float2 y = unpack2<BF16>(bw[k]);
+                    acc = fmaf(x.x, y.x, acc);
+                    acc = fmaf(x.y, y.y, acc);
+                }
+                const float lse = p.lse[(size_t)bh * p.N + r];
+                l2 = (lse == -INFINITY) ? INFINITY : lse * kLog2e;
+            }
+        }
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (g == 0 && rr < rows_total) {
+            p.dvec[rr] = acc;
+            p.lse2[rr] = l2;
+        }
+    }
+}
+
+// --------------------------------------------------------------------------- convert
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_convert_kernel(const float4 *acc, uint2 *out,
+                                                             long long n_vec4, float scale) {
+    const long long nthreads = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec4; i += nthreads) {
+        const float4 a = acc[i];
+        out[i] = make_uint2(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale));
+    }
+}
+
+// --------------------------------------------------------------------------- main
+
+struct BwdParams {
+    const float *lse2;  // [BH][Npad], log2-domain LSE (+inf for padding rows)
+    const float *dvec;  // [BH][Npad]
+    float *dq_acc;      // [BH][N][D] fp32
+    const int *kv_len;
+    int N;
+    int Npad;
+    int BH;
+    int H;
+    int num_tiles;  // ceil(N / 128)
+    float scale;
+    float scale_log2;
+    int causal;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int TILE = 128 * D * 2;  // one 128-row tile of Q / K / V / dO
+    static constexpr int HALF = 128 * 128;    // one 128-byte column block of a tile
+    static constexpr int HALVES = D / 64;
+    static constexpr bool DQ_TMA = (D == 64);  // dQ drain by TMA reduce (else red.v4)
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + TILE;
+    static constexpr int OFF_Q = OFF_V + TILE;       // 2 stages
+    static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // 2 stages
+    static constexpr int OFF_DS = OFF_DO + 2 * TILE; // 128 x 128 16-bit, operand layout
+    static constexpr int OFF_DQ = OFF_DS + 32768;    // fp32 staging (d = 64 only)
+    static constexpr int DQ_BYTES = DQ_TMA ? 128 * D * 4 : 0;
+    static constexpr int OFF_LSE = OFF_DQ + DQ_BYTES;  // 2 x 512 B
+    static constexpr int OFF_DV = OFF_LSE + 1024;      // 2 x 512 B
+    static constexpr int OFF_BAR = OFF_DV + 1024;
+    static constexpr int USED = OFF_BAR + 256;
+    // d = 128 uses all 227 KB: no room for alignment slack; the kernel checks instead.
+    static constexpr int SLACK = (USED + 1024 <= 232448) ? 1024 : 0;
+    static constexpr int SMEM = USED + SLACK;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0;
+    static constexpr uint32_t COL_DP = 128;
+    static constexpr uint32_t COL_DV = 256;
+    static constexpr uint32_t COL_DK = 256 + D;
+    static constexpr uint32_t COL_DQ = (D == 64) ? 384 : 128;  // d = 128: aliases dP^T
+};
+
+struct BwdBars {
+    uint64_t kv_full;
+    uint64_t q_full[2];
+    uint64_t do_full[2];
+    uint64_t stage_empty[2];
+    uint64_t s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_empty, dkv_full;
+    uint32_t tmem_base;
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(320, 1)
+fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+              const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+              const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad > (uint32_t)C::SLACK) {  // cannot happen with a 1024-aligned dynamic base
+        if (threadIdx.x == 0) atomicExch(&g_status, 5);
+        return;
+    }
+    uint8_t *smem = smem_raw + pad;
+    uint8_t *sK = smem + C::OFF_K;
+    uint8_t *sV = smem + C::OFF_V;
+    uint8_t *sQ = smem + C::OFF_Q;
+    uint8_t *sdO = smem + C::OFF_DO;
+    uint8_t *sdS = smem + C::OFF_DS;
+    uint8_t *sDQ = smem + C::OFF_DQ;
+    float *sLSE = reinterpret_cast<float *>(smem + C::OFF_LSE);
+    float *sDv = reinterpret_cast<float *>(smem + C::OFF_DV);
+    BwdBars *bars = reinterpret_cast<BwdBars *>(smem + C::OFF_BAR);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: key tile kt of head bh; heavier causal tiles (small kt) first.
+    const int kt = blockIdx.x / p.BH;
+    const int bh = blockIdx.x - kt * p.BH;
+    const int b = bh / p.H;
+    int L = p.N;
+    if (p.kv_len != nullptr) {
+        L = p.kv_len[b];
+        L = L < 0 ? 0 : (L > p.N ? p.N : L);
+    }
+    const int q_begin = p.causal ? kt : 0;
+    const int n = (kt * 128 < L) ? (p.num_tiles - q_begin) : 0;  // query tiles visited
+
+    if (threadIdx.x == 128) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmdO);
+        tma_prefetch_desc(&tmdK);
+        tma_prefetch_desc(&tmdV);
+        if (C::DQ_TMA) tma_prefetch_desc(&tmdQacc);
+        mbar_init(&bars->kv_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->q_full[i], 1);
+            mbar_init(&bars->do_full[i], 1);
+            mbar_init(&bars->stage_empty[i], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->ds_full, 128);
+        mbar_init(&bars->ds_empty, 1);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_empty, 128);
+        mbar_init(&bars->dkv_full, 1);
+        fence_mbar_init();
+    }
+    if (warp == 5) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0 && n > 0) {
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
+            for (int hf = 0; hf < C::HALVES; ++hf) {
+                tma_load_3d(sK + hf * C::HALF, &tmK, &bars->kv_full, hf * 64, kt * 128, bh);
+                tma_load_3d(sV + hf * C::HALF, &tmV, &bars->kv_full, hf * 64, kt * 128, bh);
+            }
+            for (int i = 0; i < n; ++i) {
+                const int s = i & 1;
+                const int qi = q_begin + i;
+                if (i >= 2 && !mbar_wait(&bars->stage_empty[s], ((i >> 1) - 1) & 1)) break;
+                const size_t vec_off = (size_t)bh * p.Npad + (size_t)qi * 128;
+                mbar_arrive_expect_tx(&bars->q_full[s], C::TILE + 512);
+                for (int hf = 0; hf < C::HALVES; ++hf)
+                    tma_load_3d(sQ + s * C::TILE + hf * C::HALF, &tmQ, &bars->q_full[s], hf * 64,
+                                qi * 128, bh);
+                bulk_load(sLSE + s * 128, p.lse2 + vec_off, 512, &bars->q_full[s]);
+                mbar_arrive_expect_tx(&bars->do_full[s], C::TILE + 512);
+                for (int hf = 0; hf < C::HALVES; ++hf)
+                    tma_load_3d(sdO + s * C::TILE + hf * C::HALF, &tmdO, &bars->do_full[s],
+                                hf * 64, qi * 128, bh);
+                bulk_load(sDv + s * 128, p.dvec + vec_off, 512, &bars->do_full[s]);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0 && n > 0) {
+            constexpr uint32_t kIdescSq = idesc_f16(BF16, false, false, 128, 128);  // S^T, dP^T
+            constexpr uint32_t kIdescTs = idesc_f16(BF16, false, true, 128, D);     // dV, dK
+            constexpr uint32_t kIdescDq = idesc_f16(BF16, true, true, 128, D);      // dQ
+            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO);
+            const uint32_t ds_addr = smem_u32(sdS);
+            // X^T = A B^T with A, B both [128 rows][D] K-major tiles.
+            auto mma_square = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * C::HALF + (kk & 3) * 32);
+                    mma_ss(d_tmem, smem_desc_sw128(a_base + off, 16, 1024),
+                           smem_desc_sw128(b_base + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+                }
+            };
+            // D[128 x D] (+)= A_tmem[128 x 128] * B[128 rows][D] (MN-major B).
+            auto mma_tmem_a = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(d_tmem, a_tmem + kk * 8,
+                           smem_desc_sw128(b_base + kk * 2048, C::HALF, 1024), kIdescTs,
+                           (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(&bars->kv_full, 0);
+            ok = ok && mbar_wait(&bars->q_full[0], 0);
+            tc_fence_after();
+            if (ok) {
+                mma_square(tmem + C::COL_S, k_addr, q_addr);
+                mma_commit(&bars->s_full);
+                ok = mbar_wait(&bars->do_full[0], 0);
+                tc_fence_after();
+            }
+            if (ok) {
+                mma_square(tmem + C::COL_DP, v_addr, do_addr);
+                mma_commit(&bars->dp_full);
+            }
+            for (int i = 0; ok && i < n; ++i) {
+                const int s = i & 1;
+                if (!mbar_wait(&bars->p_full, i & 1)) break;
+                tc_fence_after();
+                mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_S, do_addr + s * C::TILE, i > 0);
+                if (i + 1 < n) {
+                    const int s1 = (i + 1) & 1;
+                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
+                    tc_fence_after();
+                    mma_square(tmem + C::COL_S, k_addr, q_addr + s1 * C::TILE);
+                    mma_commit(&bars->s_full);
+                }
+                if (!mbar_wait(&bars->ds_full, i & 1)) break;
+                tc_fence_after();
+                mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, q_addr + s * C::TILE, i > 0);
+                if (D == 64 && i > 0) {
+                    if (!mbar_wait(&bars->dq_empty, (i - 1) & 1)) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + C::COL_DQ, smem_desc_sw128(ds_addr + kk * 2048, 16384, 1024),
+                           smem_desc_sw128(k_addr + kk * 2048, C::HALF, 1024), kIdescDq,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(&bars->dq_full);
+                mma_commit(&bars->ds_empty);
+                mma_commit(&bars->stage_empty[s]);
+                if (i + 1 < n) {
+                    const int s1 = (i + 1) & 1;
+                    if (D == 128) {
+                        // dQ_i lives in the dP^T columns: wait until it has been drained.
+                        if (!mbar_wait(&bars->dq_empty, i & 1)) break;
+                    }
+                    if (!mbar_wait(&bars->do_full[s1], ((i + 1) >> 1) & 1)) break;
+                    tc_fence_after();
+                    mma_square(tmem + C::COL_DP, v_addr, do_addr + s1 * C::TILE);
+                    mma_commit(&bars->dp_full);
+                }
+            }
+            mma_commit(&bars->dkv_full);
+        }
+    } else if (warp >= 6) {
+        // ------------------------------ dQ drain ----------------------------------
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;  // query row in the tile = TMEM lane
+        const int gt = threadIdx.x - 192;   // 0..127 inside this warpgroup
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        for (int i = 0; i < n; ++i) {
+            const int qi = q_begin + i;
+            if (!mbar_wait(&bars->dq_full, i & 1)) break;
+            tc_fence_after();
+            float v[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t w[32];
+                tmem_ld32(tmem + lane_base + C::COL_DQ + c * 32, w);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[c * 32 + k] = __uint_as_float(w[k]);
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->dq_empty);
+            if constexpr (C::DQ_TMA) {
+                if (gt == 0) bulk_wait_group_read<0>();
+                named_bar_sync(2, 128);
+                // D/32 boxes of [128 rows][32 fp32], 16-byte chunks swizzled by row % 8.
+#pragma unroll
+                for (int bx = 0; bx < D / 32; ++bx) {
+                    uint8_t *rowp = sDQ + bx * 16384 + r * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float *x = v + bx * 32 + c * 4;
+                        *reinterpret_cast<float4 *>(rowp + ((c ^ (r & 7)) << 4)) =
+                            make_float4(x[0], x[1], x[2], x[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(2, 128);
+                if (gt == 0) {
+#pragma unroll
+                    for (int bx = 0; bx < D / 32; ++bx)
+                        tma_reduce_add_3d(&tmdQacc, sDQ + bx * 16384, bx * 32, qi * 128, bh);
+                    bulk_commit_group();
+                }
+            } else {
+                const int row = qi * 128 + r;
+                if (row < p.N) {
+                    float *dst = p.dq_acc + ((size_t)bh * p.N + row) * D;
+#pragma unroll
+                    for (int c = 0; c < D; c += 4) red_add_v4(dst + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+                }
+            }
+        }
+        if constexpr (C::DQ_TMA) {
+            if (gt == 0) bulk_wait_group<0>();
+        }
+    } else {
+        // ------------------------------ P / dS warps ------------------------------
+        const int t = threadIdx.x;  // key row in the tile = TMEM lane
+        const int key = kt * 128 + t;
+        const bool key_ok = key < L;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int i = 0; i < n; ++i) {
+            const int s = i & 1;
+            const int qi = q_begin + i;
+            if (!mbar_wait(&bars->s_full, i & 1) || !mbar_wait(&bars->q_full[s], (i >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // P^T row, kept as packed 16-bit pairs (exactly what the dV MMA consumes);
+            // dS below uses the same rounded values.
+            uint32_t Pw[64];
+            const float *lse2 = sLSE + s * 128;
+            const bool diag = p.causal && (qi == kt);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t w[32];
+                tmem_ld32(tmem + lane_base + C::COL_S + cc * 32, w);
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                    const int c = cc * 32 + k;
+                    const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + c);
+                    float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
+                    float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
+                    float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
+                    float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
+                    // masked: keys past the valid length, queries before the key (causal)
+                    if (!key_ok || (diag && c < t)) p0 = 0.f;
+                    if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
+                    if (!key_ok || (diag && c + 2 < t)) p2 = 0.f;
+                    if (!key_ok || (diag && c + 3 < t)) p3 = 0.f;
+                    Pw[c >> 1] = pack2<BF16>(p0, p1);
+                    Pw[(c >> 1) + 1] = pack2<BF16>(p2, p3);
+                }
+            }
+            {
+                uint32_t w[32];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) w[k] = Pw[h * 32 + k];
+                    tmem_st32(tmem + lane_base + C::COL_S + h * 32, w);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+
+            if (!mbar_wait(&bars->dp_full, i & 1) || !mbar_wait(&bars->do_full[s], (i >> 1) & 1) ||
+                (i > 0 && !mbar_wait(&bars->ds_empty, (i - 1) & 1))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float *dv = sDv + s * 128;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t w[32];
+                tmem_ld32(tmem + lane_base + C::COL_DP + cc * 32, w);
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) {
+                    const int c = cc * 32 + k;
+                    const float2 d2 = *reinterpret_cast<const float2 *>(dv + c);
+                    const float2 pp = unpack2<BF16>(Pw[c >> 1]);
+                    const float ds0 = pp.x * (__uint_as_float(w[k]) - d2.x);
+                    const float ds1 = pp.y * (__uint_as_float(w[k + 1]) - d2.y);
+                    pk[k >> 1] = pack2<BF16>(ds0, ds1);
+                }
+                // dS^T row -> TMEM (columns already read), A operand of dK += dS^T Q.
+                tmem_st16(tmem + lane_base + C::COL_DP + cc * 16, pk);
+                // dS -> shared memory as the MN-major A operand of dQ = dS K:
+                // [query block (64)][key row t][64 queries], 128-byte swizzle.
+                uint8_t *rowp = sdS + (cc >> 1) * 16384 + t * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int chunk = (cc & 1) * 4 + q4;
+                    *reinterpret_cast<uint4 *>(rowp + ((chunk ^ (t & 7)) << 4)) =
+                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_full);
+        }
+
+        // ------------------------------ epilogue: dK, dV ------------------------------
+        if (ok && n > 0) {
+            ok = mbar_wait(&bars->dkv_full, 0);
+            tc_fence_after();
+        }
+        // Staging: the first Q / dO stage buffers are free once every MMA is done.
+        uint8_t *stage_v = sQ;
+        uint8_t *stage_k = sdO;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const uint32_t col = which == 0 ? C::COL_DV : C::COL_DK;
+            const float mul = which == 0 ? 1.f : p.scale;
+            uint8_t *stage = which == 0 ? stage_v : stage_k;
+#pragma unroll
+            for (int hf = 0; hf < C::HALVES; ++hf) {
+                uint32_t wv[32];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t w[32];
+                    if (n > 0) {
+                        tmem_ld32(tmem + lane_base + col + hf * 64 + h2 * 32, w);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) w[k] = 0u;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        wv[h2 * 16 + k] = pack2<BF16>(__uint_as_float(w[2 * k]) * mul,
+                                                      __uint_as_float(w[2 * k + 1]) * mul);
+                }
+                uint8_t *rowp = stage + hf * C::HALF + t * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(rowp + ((c ^ (t & 7)) << 4)) =
+                        make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+            }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (t == 0) {
+            for (int hf = 0; hf < C::HALVES; ++hf) {
+                tma_store_3d(&tmdV, stage_v + hf * C::HALF, hf * 64, kt * 128, bh);
+                tma_store_3d(&tmdK, stage_k + hf * C::HALF, hf * 64, kt * 128, bh);
+            }
+            bulk_commit_group();
+            bulk_wait_group_read<0>();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace fa
