@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one forward pass and one backward pass of the whole path over one batch of
+the GPT-2-small shaped workload (B8 H12 N1024 d64 bf16, causal), seeded synthetic data.
+The metric is attention forward+backward TFLOP/s with the nominal FLOP count
+(4 B H N^2 d forward, 2.5x that backward, halved for causal).  Prints ONE JSON line.
+
+Multi-GPU (one process per GPU under torchrun): every rank runs its own batch (weak
+scaling); the heads are independent, so there is no data-path collective; the timed
+region is bracketed by barriers and the reported time is the maximum over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (test infrastructure) on the host cores,
+each step one bounded sample of the same workload; only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, 1×B200) and % of dense tensor-core peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "gpt2"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+REASON_FIELDS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+# ------------------------------------------------------------------ host-side helpers
+# (kept free of CUDA so that the multi-rank logic is testable with gloo on CPU)
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling)."""
+    return 1000 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def step_flops(w) -> tuple:
+    f, b = w.nominal_flops()
+    return f, b, f + b
+
+
+def whole_job_tflops(flops_per_step: float, n_gpus: int, steps: int, max_ms: float) -> float:
+    return n_gpus * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_60_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of ``kernel`` from the committed ncu summary, if that summary
+    was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
+    try:
+        with open(path) as f:
+            txt = f.read()
+    except OSError:
+        return None
+    vals = {}
+    for line in txt.splitlines():
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha") != kernel_source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons of one GPU in the background."""
+
+    QUERY = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[3], parts[5:9]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        note = "samples inside the timed region"
+        if not inside:
+            inside = rows
+            note = "timed region shorter than the sampling period: samples of the whole run"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+        reasons = set()
+        for r in inside:
+            for name, val in zip(REASON_FIELDS, r[4]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "note": note}
+
+
+def gpu_pci_id(dev: int) -> str:
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except AttributeError:
+        return str(dev)
+
+
+# ------------------------------------------------------------------ our arm
+
+def alloc_set(w, inp, dev):
+    import torch
+    from exact_io_aware_60_b200 import fa
+    s = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
+    s["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
+    s["o"] = torch.empty_like(s["q"])
+    s["lse"] = torch.empty(s["q"].shape[:-1], dtype=torch.float32, device=dev)
+    s["dq"], s["dk"], s["dv"] = (torch.empty_like(s["q"]) for _ in range(3))
+    s["ws"] = fa.workspace_for(s["q"])
+    return s
+
+
+def set_bytes(s) -> int:
+    return sum(t.numel() * t.element_size() for n, t in s.items() if t is not None)
+
+
+def run_step(w, s, stream=None):
+    from exact_io_aware_60_b200 import fa
+    fa.fa_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale, causal=w.causal,
+              kv_len=s["kv_len"], stream=stream)
+    fa.fa_bwd(s["q"], s["k"], s["v"], s["o"], s["do"], s["lse"], s["dq"], s["dk"], s["dv"],
+              scale=w.scale, causal=w.causal, kv_len=s["kv_len"], workspace=s["ws"],
+              stream=stream)
+
+
+def cpu_baseline_sample(w, inp, budget_s: float) -> dict:
+    """The oracle (as it stands) on whole heads of the workload until ``budget_s`` of CPU
+    time has passed (at least one head)."""
+    import oracle
+    q, k, v, do = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    t0 = time.perf_counter()
+    done = 0
+    for b, h in heads:
+        L = w.N if kv is None else int(kv[b])
+        oracle.attention_rows(q[b, h], k[b, h], v[b, h], do[b, h], scale=w.scale,
+                              causal=w.causal, kv_len=L)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = step_flops(w)[2] * done / (w.B * w.H)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"fp64 oracle forward+backward of {done} of {w.B * w.H} (batch, head) "
+                      f"pairs of the {w.name} workload in {dt:.1f} s (nominal FLOPs)"}
+
+
+def bench_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_60_b200 import fa
+    from exact_io_aware_60_b200 import workloads as W
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.workload]
+    f_fwd, f_bwd, f_step = step_flops(w)
+
+    inp = W.make_inputs(w, seed=rank_seed(rank))
+    first = alloc_set(w, inp, dev)
+    per_set = set_bytes(first)
+    l2 = 126 * 2 ** 20
+    nsets = max(2, math.ceil(2 * l2 / per_set) + 1)
+    sets = [first] + [alloc_set(w, W.make_inputs(w, seed=rank_seed(rank) + i), dev)
+                      for i in range(1, nsets)]
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for i in range(args.warmup):
+        run_step(w, sets[i % nsets])
+    torch.cuda.synchronize(dev)
+    status = fa.fa_get_device_status()
+    if status != fa.FA_OK:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    # per-kernel events (forward kernel, backward main kernel), one pair per launch
+    K = args.steps
+    evs = {0: [], 1: []}
+    for which in (0, 1):
+        for _ in range(K):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            b.record(stream)
+            evs[which].append((a, b))
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_pci_id(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark("t0")
+    start.record(stream)
+    for i in range(K):
+        fa.fa_set_timing_events(0, *evs[0][i])
+        fa.fa_set_timing_events(1, *evs[1][i])
+        run_step(w, sets[i % nsets])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark("t1")
+    barrier()
+    torch.cuda.synchronize(dev)
+    fa.fa_set_timing_events(0)
+    fa.fa_set_timing_events(1)
+    clk = clocks.stop()
+    status = fa.fa_get_device_status()
+    if status != fa.FA_OK:
+        raise RuntimeError(f"device status {status} after the timed region")
+    ms = start.elapsed_time(end)
+    max_ms = max_over_ranks(ms, dev if world > 1 else None)
+    k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / K
+    k_bwd = sum(a.elapsed_time(b) for a, b in evs[1]) / K
+    value = whole_job_tflops(f_step, world, K, max_ms)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
+        outs = {n: torch.empty(first[n].shape, dtype=first[n].dtype, pin_memory=True)
+                for n in ("o", "lse", "dq", "dk", "dv")}
+        Ke = max(3, min(K, args.e2e_steps))
+        s = first
+
+        def e2e_step():
+            for n in ("q", "k", "v", "do"):
+                s[n].copy_(host[n], non_blocking=True)
+            run_step(w, s)
+            for n in ("o", "lse", "dq", "dk", "dv"):
+                outs[n].copy_(s[n], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = max_over_ranks(a.elapsed_time(b), dev if world > 1 else None)
+        e2e = {"value": whole_job_tflops(f_step, world, Ke, e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs.values()),
+               "steps": Ke, "ms_per_step": e_ms / Ke}
+
+    peaks, peak_src = load_peaks()
+    sustained = ms > 1000.0
+    peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    # the dominant kernel is the one with the larger device time per step
+    if k_bwd >= k_fwd:
+        dom_name, dom_flops, dom_ms = "fa_bwd_kernel", f_bwd, k_bwd
+    else:
+        dom_name, dom_flops, dom_ms = "fa_fwd_kernel", f_fwd, k_fwd
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peak_src} {peak_key}",
+                "flops_per_launch": dom_flops, "launch_ms": dom_ms,
+                "traffic": profile_traffic(dom_name, w.name)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(w, inp, args.cpu_seconds)
+
+    per_rank_value = f_step * K / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16"}[w.dtype],
+        "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
+        "config": {"workload": w.description + ", forward + backward", "B": w.B, "H": w.H,
+                   "N": w.N, "d": w.d, "causal": w.causal,
+                   "flops_per_step": f_step, "parallelism": f"replicas x{world} (no collective)",
+                   "l2": f"{nsets} resident input/output sets ({nsets * per_set / 2**20:.0f} MiB) "
+                         "rotated so each step reads data evicted from the 126 MB L2"},
+        "pct_of_peak": 100.0 * per_rank_value / peak,
+        "kernels": {"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12},
+                    "fa_bwd_kernel": {"ms": k_bwd, "tflops": f_bwd / (k_bwd * 1e-3) / 1e12}},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 4 * K,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+    return line
+
+
+# ------------------------------------------------------------------ reference arm
+
+def bench_reference(args):
+    """The fp64 oracle on the host cores; each step is one bounded sample of the workload
+    (the forward + backward of one (batch, head) pair, or of a row subset of it when the
+    requested step count would not finish within a few minutes)."""
+    import numpy as np
+    import oracle
+    from exact_io_aware_60_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(w, seed=0)
+    q, k, v, do = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    total = args.steps + args.warmup
+    rows_per_step = w.N if total <= 300 else max(16, (w.N * 300) // total)
+    rng = np.random.default_rng(0)
+
+    def flops_of(rows, L):
+        vis = 0
+        for i in rows:
+            vis += min(L, i + 1) if w.causal else L
+        return 14.0 * w.d * vis  # 4d forward + 10d backward per visible score
+
+    def one(i):
+        b, h = heads[i % len(heads)]
+        L = w.N if kv is None else int(kv[b])
+        rows = (np.arange(w.N) if rows_per_step >= w.N
+                else np.sort(rng.choice(w.N, rows_per_step, replace=False)))
+        oracle.attention_rows(q[b, h], k[b, h], v[b, h], do[b, h], scale=w.scale,
+                              causal=w.causal, kv_len=L, rows=rows)
+        return flops_of(rows, L)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    fl = 0.0
+    for i in range(args.steps):
+        fl += one(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = fl / dt / 1e12
+    sample = (f"fp64 oracle forward+backward of {rows_per_step} query rows of one (batch, head) "
+              f"pair per step, {w.name} workload")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
+        "config": {"workload": w.description + ", forward + backward", "B": w.B, "H": w.H,
+                   "N": w.N, "d": w.d, "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(bench_reference(args)), flush=True)
+        return 0
+    line = bench_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

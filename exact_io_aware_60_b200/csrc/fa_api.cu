@@ -23,6 +23,12 @@ constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxDevices = 64;
 
 thread_local char t_last_error[256] = "";
+thread_local cudaEvent_t t_timing[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+
+// Records the profiling event of `which` (0 fwd, 1 bwd main), side 0 before / 1 after.
+void timing_mark(int which, int side, cudaStream_t st) {
+    if (t_timing[which][side] != nullptr) cudaEventRecord(t_timing[which][side], st);
+}
 
 void record_cuda_error(cudaError_t e, const char *where) {
     snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
@@ -150,8 +156,10 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     }
     const long long grid = (long long)p.num_q_tiles * bh;
     if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    timing_mark(0, 0, st);
     kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
     e = cudaGetLastError();
+    timing_mark(0, 1, st);
     if (e != cudaSuccess) {
         record_cuda_error(e, "fa_fwd launch");
         return FA_ERR_CUDA;
@@ -254,8 +262,10 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     }
     const long long grid = (long long)num_tiles * bh;
     if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    timing_mark(1, 0, st);
     kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
     e = cudaGetLastError();
+    timing_mark(1, 1, st);
     if (e != cudaSuccess) {
         record_cuda_error(e, "fa_bwd launch");
         return FA_ERR_CUDA;
@@ -278,6 +288,14 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 extern "C" {
 
 int fa_version(void) { return kVersion; }
+
+int fa_set_timing_events(int which, void *start, void *stop) {
+    if (which < 0 || which > 1) return FA_ERR_INVALID_ARG;
+    if ((start == nullptr) != (stop == nullptr)) return FA_ERR_INVALID_ARG;
+    t_timing[which][0] = reinterpret_cast<cudaEvent_t>(start);
+    t_timing[which][1] = reinterpret_cast<cudaEvent_t>(stop);
+    return FA_OK;
+}
 
 const char *fa_strerror(int status) {
     switch (status) {
@@ -341,6 +359,21 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
         return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
     return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
 #undef FA_BWD_ARGS
+}
+
+int fa_selftest_wait_timeout(int limit_us, void *stream) {
+    if (limit_us < 1 || limit_us > 2000000) return FA_ERR_INVALID_ARG;
+    int dev = 0;
+    int rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    fa::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)limit_us * 1000ull);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "selftest launch");
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
 }
 
 int fa_get_device_status(void *stream) {

@@ -18,8 +18,13 @@
 //               MUFU ex2, row sum, P_j written back into TMEM as 16-bit pairs over S_j.
 //               The output rescale is lazy: m only moves when the row max grows by more
 //               than 2^8, which leaves the result exact because O and l always share the
-//               same m.  Epilogue: O / l -> 16-bit, staged swizzled in shared memory and
+//               same m.  Epilogue: O / l' -> 16-bit, staged swizzled in shared memory and
 //               written with one TMA store; LSE = ln2 * (m + log2 l).
+//   Normaliser: the tensor core multiplies V by P rounded to 16 bits, so the output is
+//   divided by l' = sum of exactly those rounded values, produced by one more small MMA
+//   (P times a tile of ones) into 16 spare TMEM columns.  The weights applied to the rows
+//   of V then sum to one exactly, which removes the bias a fp32 l would leave when one
+//   key dominates a row.  LSE keeps the fp32 sum l of the unrounded values.
 // The loop order is query-block outer (each CTA writes its O rows once) instead of the
 // key-block-outer order of the original algorithm; the result is the same up to
 // floating-point ordering.
@@ -53,11 +58,13 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + TILE;
     static constexpr int OFF_V = OFF_K + NS * TILE;
-    static constexpr int OFF_BAR = OFF_V + NS * TILE;
+    static constexpr int OFF_ONES = OFF_V + NS * TILE;   // 2 KB of 16-bit ones
+    static constexpr int OFF_BAR = OFF_ONES + 2048;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;   // + barriers + alignment slack
     static constexpr int THREADS = 192;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = 256;              // S0 at 0, S1 at 128, O at 256
+    static constexpr uint32_t COL_SUM = 256 + D;        // 16 columns: row sums of 16-bit P
 };
 
 struct FwdBars {
@@ -120,6 +127,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         fence_mbar_init();
     }
+    if (warp == 4) {
+        // 16-bit ones: B operand of the row-sum MMA (layout-agnostic: every element is 1)
+        const uint32_t one2 = BF16 ? 0x3F803F80u : 0x3C003C00u;
+        uint32_t *ones = reinterpret_cast<uint32_t *>(smem + C::OFF_ONES);
+        for (int i = lane; i < 512; i += 32) ones[i] = one2;
+        fence_proxy_async_smem();
+    }
     if (warp == 5) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
@@ -150,6 +164,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (lane == 0 && T > 0) {
             constexpr uint32_t kIdescS = idesc_f16(BF16, false, false, 128, 128);
             constexpr uint32_t kIdescO = idesc_f16(BF16, false, true, 128, D);
+            constexpr uint32_t kIdescSum = idesc_f16(BF16, false, false, 128, 16);
+            const uint64_t ones_desc = smem_desc_sw128(smem_u32(smem + C::OFF_ONES), 16, 1024);
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t k_addr = smem_u32(sK);
             const uint32_t v_addr = smem_u32(sV);
@@ -185,6 +201,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mma_ts(tmem + C::COL_O, p_tmem + kk * 8, bd, kIdescO,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    mma_ts(tmem + C::COL_SUM, p_tmem + kk * 8, ones_desc, kIdescSum,
+                           (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bars->kv_empty[s]);
                 mma_commit(&bars->o_full);
             }
@@ -276,6 +296,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
                     tmem_st32(ob + c * 32, r);
                 }
+                {
+                    uint32_t r[16];
+                    tmem_ld16(ob + D, r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st16(ob + D, r);
+                }
             }
             tc_fence_before();
             mbar_arrive(&bars->p_full[j & 1]);
@@ -286,8 +313,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             ok = mbar_wait(&bars->o_full, (T - 1) & 1);
             tc_fence_after();
         }
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
         const uint32_t ob = tmem + lane_base + C::COL_O;
+        float l_round = 0.f;
+        if (T > 0) {
+            uint32_t r[16];
+            tmem_ld16(ob + D, r);
+            l_round = __uint_as_float(r[0]);
+        }
+        const float inv = (l > 0.f && l_round > 0.f) ? 1.f / l_round : 0.f;
 #pragma unroll
         for (int hf = 0; hf < C::HALVES; ++hf) {
             uint32_t w[32];

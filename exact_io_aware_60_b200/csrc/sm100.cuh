@@ -68,17 +68,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity of `bar` has completed.  Returns false
-// (after recording FA_ERR_TIMEOUT = 4 in g_status) if the deadline passes first.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// (after recording FA_ERR_TIMEOUT = 4 in g_status) if `limit_ns` passes first.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity,
+                                                uint64_t limit_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(a, parity)) return true;
-        if ((it & 63u) == 0u && globaltimer() - t0 > kWaitLimitNs) {
+        if ((it & 63u) == 0u && globaltimer() - t0 > limit_ns) {
             atomicExch(&g_status, 4);
             return false;
         }
+    }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    return mbar_wait_limit(bar, parity, kWaitLimitNs);
+}
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing will ever
+// complete.  The wait must give up after `limit_ns` and record the timeout status;
+// nothing else is held (no TMEM, no copies in flight), so the kernel always returns.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        (void)mbar_wait_limit(&bar, 0, limit_ns);
     }
 }
 
@@ -260,6 +277,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
         "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
         "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// TMEM -> registers, 32 lanes x 16 consecutive 32-bit columns; waits for completion.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
         : "memory");
 }
 

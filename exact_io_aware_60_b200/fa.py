@@ -65,6 +65,10 @@ def lib():
             L.fa_get_device_status.argtypes = [vp]
             L.fa_version.restype = i
             L.fa_version.argtypes = []
+            L.fa_set_timing_events.restype = i
+            L.fa_set_timing_events.argtypes = [i, vp, vp]
+            L.fa_selftest_wait_timeout.restype = i
+            L.fa_selftest_wait_timeout.argtypes = [i, vp]
             _lib = L
     return _lib
 
@@ -147,6 +151,24 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: bool = Fa
                       workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
+
+
+def fa_set_timing_events(which: int, start=None, stop=None) -> None:
+    """Profiling hook: record torch.cuda.Event ``start``/``stop`` around every launch of
+    the forward kernel (which=0) or the backward main kernel (which=1); None switches it
+    off.  The events must have been recorded once (so that they exist)."""
+    h0 = None if start is None else start.cuda_event
+    h1 = None if stop is None else stop.cuda_event
+    rc = lib().fa_set_timing_events(int(which), h0, h1)
+    if rc != FA_OK:
+        raise FAError(rc, "fa_set_timing_events")
+
+
+def fa_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueues the bounded-wait self-test kernel (see include/fa.h)."""
+    rc = lib().fa_selftest_wait_timeout(int(limit_us), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_selftest_wait_timeout")
 
 
 def fa_get_device_status(stream=None) -> int:

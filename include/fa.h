@@ -90,8 +90,8 @@ FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *l
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 [B, H, N, d] dQ
- * accumulator and an fp32 [B, H, N] array D_i = sum_c dO_ic O_ic, each 256-byte
- * aligned.  Returns 0 for invalid sizes.
+ * accumulator, then two fp32 [B, H, ceil(N/128)*128] arrays (D_i = sum_c dO_ic O_ic
+ * and the log-sum-exp in base 2), each 256-byte aligned.  Returns 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -126,6 +126,26 @@ FA_API const char *fa_last_cuda_error(void);
  * last call, or FA_ERR_CUDA if the synchronisation failed.
  */
 FA_API int fa_get_device_status(void *stream);
+
+/*
+ * Optional timing hook for profiling.  After this call, every launch made by this host
+ * thread of the selected kernel records `start` on the launch stream immediately
+ * before the kernel and `stop` immediately after it, so cudaEventElapsedTime(start,
+ * stop) is that kernel's device time.  which = 0: the forward kernel of fa_fwd;
+ * which = 1: the main kernel of fa_bwd (not its preprocess and convert kernels).
+ * start, stop: cudaEvent_t handles created by the caller, or both NULL to switch the
+ * hook off.  Returns FA_OK or FA_ERR_INVALID_ARG.
+ */
+FA_API int fa_set_timing_events(int which, void *start, void *stop);
+
+/*
+ * Self-test of the bounded device waits: enqueues one kernel whose single thread waits
+ * on a barrier that nothing ever completes, with a limit of `limit_us` microseconds
+ * (1 .. 2000000).  The wait gives up and records FA_ERR_TIMEOUT in the device status
+ * word, exactly as a stalled wait inside fa_fwd / fa_bwd would; the CUDA context stays
+ * usable.  Returns FA_OK once enqueued.
+ */
+FA_API int fa_selftest_wait_timeout(int limit_us, void *stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 FA_API int fa_version(void);

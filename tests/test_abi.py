@@ -41,8 +41,9 @@ def test_version_and_strerror():
 def test_workspace_bytes():
     L = fa.lib()
     n = L.fa_bwd_workspace_bytes(2, 3, 100, 64)
-    rows = 2 * 3 * 100
-    assert n == ((rows * 64 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    r256 = lambda x: ((x + 255) // 256) * 256
+    # fp32 dQ accumulator [B,H,N,d] + two fp32 [B,H,Npad] vectors (Npad = 128)
+    assert n == r256(2 * 3 * 100 * 64 * 4) + 2 * r256(2 * 3 * 128 * 4)
     assert L.fa_bwd_workspace_bytes(0, 3, 100, 64) == 0
 
 
@@ -95,6 +96,13 @@ def call_bwd(**over):
 ])
 def test_bwd_rejects_bad_arguments_on_host(over, code):
     assert call_bwd(**over) == code
+
+
+def test_timing_hook_arguments():
+    L = fa.lib()
+    assert L.fa_set_timing_events(2, None, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_set_timing_events(0, P, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_set_timing_events(1, None, None) == fa.FA_OK
 
 
 def test_binding_raises_without_cuda_tensors():

@@ -1,0 +1,94 @@
+"""bench.py host logic without a GPU: the max-over-ranks timing with 2 gloo ranks, the
+weak-scaling aggregate, the oracle reference arm and the stale-profile check."""
+import io
+import json
+import os
+import socket
+import contextlib
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t = bench.max_over_ranks(10.0 + 5.0 * rank)
+        seed = bench.rank_seed(rank)
+        q.put((rank, t, seed))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [r[1] for r in res] == [15.0, 15.0]      # every rank sees the slowest time
+    assert res[0][2] != res[1][2]                    # each rank draws its own batch
+
+
+def test_whole_job_value_is_weak_scaling_aggregate():
+    f = 1e12
+    assert bench.whole_job_tflops(f, 1, 10, 1000.0) == pytest.approx(10.0)
+    assert bench.whole_job_tflops(f, 4, 10, 1000.0) == pytest.approx(40.0)
+
+
+def test_reference_arm_prints_one_json_line():
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3",
+                         "--workload", "tiny"])
+    assert rc == 0
+    lines = [l for l in buf.getvalue().splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_do_nothing(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    assert buf.getvalue() == ""
+
+
+def test_warmup_minimum():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
+
+
+def test_profile_traffic_only_for_current_sources(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    csrc = tmp_path / "exact_io_aware_60_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cuh").write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    sha = bench.kernel_source_sha()
+    (tmp_path / "profiles" / "fa_bwd_kernel_gpt2.txt").write_text(
+        f"source_sha: {sha}\ndram_bytes_per_launch: 12345\n")
+    assert bench.profile_traffic("fa_bwd_kernel", "gpt2") == 12345.0
+    (csrc / "k.cuh").write_text("kernel v2")
+    assert bench.profile_traffic("fa_bwd_kernel", "gpt2") is None
