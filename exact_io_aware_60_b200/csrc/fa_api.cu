@@ -283,6 +283,28 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     return FA_OK;
 }
 
+// Static scratch of fa_bwd_noalloc.  In host code this name is only a stand-in for the
+// device symbol: its device address is looked up with cudaGetSymbolAddress (once per
+// device, with that device current) and that address is what the kernels get.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+std::atomic<void *> g_noalloc_ptr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on device `dev` (which must be current).
+int noalloc_scratch(int dev, void **out) {
+    void *p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            record_cuda_error(e, "cudaGetSymbolAddress(noalloc scratch)");
+            return FA_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -304,6 +326,7 @@ const char *fa_strerror(int status) {
         case FA_ERR_UNSUPPORTED: return "unsupported configuration or device";
         case FA_ERR_CUDA: return "CUDA error";
         case FA_ERR_TIMEOUT: return "device-side wait timed out";
+        case FA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than fa_bwd_noalloc's static buffer";
         default: return "unknown status";
     }
 }
@@ -374,6 +397,32 @@ int fa_selftest_wait_timeout(int limit_us, void *stream) {
         return FA_ERR_CUDA;
     }
     return FA_OK;
+}
+
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                   const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+                   float scale, int causal, const int *kv_len, int dtype, void *stream) {
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_INVALID_ARG;
+    if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, N, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    if (fa_bwd_workspace_bytes(B, H, N, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
+    int dev = 0;
+    rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    void *workspace = nullptr;
+    rc = noalloc_scratch(dev, &workspace);
+    if (rc != FA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, workspace, st, dev
+    if (d == 64)
+        return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
+    return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
+#undef FA_BWD_ARGS
 }
 
 int fa_get_device_status(void *stream) {

@@ -21,6 +21,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_ERR_SCRATCH_LIMIT = 5
+FA_NOALLOC_SCRATCH_BYTES = 64 << 20
 FA_BF16, FA_FP16 = 0, 1
 
 _lock = threading.Lock()
@@ -69,6 +71,9 @@ def lib():
             L.fa_set_timing_events.argtypes = [i, vp, vp]
             L.fa_selftest_wait_timeout.restype = i
             L.fa_selftest_wait_timeout.argtypes = [i, vp]
+            L.fa_bwd_noalloc.restype = i
+            L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i,
+                                         vp, i, vp]
             _lib = L
     return _lib
 
@@ -76,7 +81,9 @@ def lib():
 def fa_strerror(status: int) -> str:
     if _lib is None:
         return {0: "ok", 1: "invalid argument", 2: "unsupported configuration or device",
-                3: "CUDA error", 4: "device-side wait timed out"}.get(status, "unknown status")
+                3: "CUDA error", 4: "device-side wait timed out",
+                5: "problem needs more scratch than fa_bwd_noalloc's static buffer"}.get(
+                    status, "unknown status")
     return _lib.fa_strerror(int(status)).decode()
 
 
@@ -151,6 +158,25 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: bool = Fa
                       workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: bool = False,
+                   kv_len=None, stream=None) -> None:
+    """Enqueues the backward pass using the library's static scratch instead of a
+    caller workspace, for callers that cannot allocate device memory (see include/fa.h:
+    problems needing more than FA_NOALLOC_SCRATCH_BYTES of scratch are refused, and
+    calls that may overlap on the GPU race on the shared scratch)."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    rc = lib().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                              _kv_ptr(kv_len, B), _dtype_code(q), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_noalloc")
 
 
 def fa_set_timing_events(which: int, start=None, stop=None) -> None:

@@ -66,7 +66,8 @@ typedef enum {
     FA_ERR_INVALID_ARG = 1,
     FA_ERR_UNSUPPORTED = 2,
     FA_ERR_CUDA = 3,
-    FA_ERR_TIMEOUT = 4
+    FA_ERR_TIMEOUT = 4,
+    FA_ERR_SCRATCH_LIMIT = 5
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -126,6 +127,45 @@ FA_API const char *fa_last_cuda_error(void);
  * last call, or FA_ERR_CUDA if the synchronisation failed.
  */
 FA_API int fa_get_device_status(void *stream);
+
+/*
+ * Backward pass for callers that cannot allocate device memory.  The FlashAttention
+ * pages have no counterpart to this entry point: it exists for the environment, not the
+ * method.  Some hosts of this library may not call cudaMalloc at all: plugins inside
+ * an inference engine or framework that owns every byte of device memory and hands its
+ * plugins no allocator, and serving loops that forbid device allocation once they have
+ * started, because cudaMalloc can synchronise the device and stall every stream.  Such
+ * callers can still provide their inputs and outputs but have nowhere to get the
+ * backward pass's scratch from.
+ *
+ * fa_bwd_noalloc computes exactly what fa_bwd computes (same arguments, same kernels,
+ * same results) but takes its scratch (the fp32 dQ accumulator and the two per-row
+ * vectors described at fa_bwd_workspace_bytes) from one static device array of
+ * FA_NOALLOC_SCRATCH_BYTES bytes inside the library.  Every GPU that loads the
+ * library holds that array until the process exits.  The entry point itself calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Limit: the call is accepted only if fa_bwd_workspace_bytes(B, H, N, d) <=
+ * FA_NOALLOC_SCRATCH_BYTES; with N a multiple of 128 that is up to B*H*N = 254080 rows
+ * at d = 64 and 129024 rows at d = 128.  Larger problems return FA_ERR_SCRATCH_LIMIT and
+ * enqueue nothing.
+ *
+ * Set-up: the first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture begins.
+ *
+ * Sharing: all calls share the one array, and it keeps the previous call's contents;
+ * the call clears what must start at zero itself.  Two calls whose kernels may overlap
+ * on the GPU (different streams without ordering, or several host threads) race on the
+ * array and produce wrong gradients: order them on one stream, or use fa_bwd with
+ * separate workspaces.
+ *
+ * Arguments, layout, ownership and the other error codes are those of fa_bwd.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                          const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                          int B, int H, int N, int d, float scale, int causal,
+                          const int *kv_len, int dtype, void *stream);
 
 /*
  * Optional timing hook for profiling.  After this call, every launch made by this host

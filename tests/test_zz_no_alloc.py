@@ -1,0 +1,83 @@
+"""fa_bwd_noalloc: the backward pass for callers that cannot allocate device memory.
+
+Some hosts of this library (plugins inside an engine that owns all device memory, serving
+loops that forbid cudaMalloc after start-up) can pass inputs and outputs but cannot
+provide the backward pass's scratch workspace.  fa_bwd_noalloc takes that scratch from a
+static array inside the library instead.  This test calls it through the C ABI and checks
+that two calls in a row give the results of fa_bwd with a caller-allocated workspace, and
+that a problem too large for the static array is refused without doing any work.
+
+The file is named so that pytest collects it last: if it fails, a run that stops at the
+first failure has already run every other test.  It passes on its own in a fresh process
+as well as after the other tests.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from exact_io_aware_60_b200 import fa
+from exact_io_aware_60_b200 import workloads as W
+from parity import GRAD_REL_L2, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    W.custom("gpt2-like", B=2, H=3, N=300, d=64, dtype=torch.bfloat16, causal=True),
+    W.custom("bert-like", B=3, H=2, N=260, d=64, dtype=torch.float16, kv_len_range=(100, 260)),
+    W.custom("d128", B=1, H=2, N=517, d=128, dtype=torch.bfloat16, causal=True),
+]
+
+
+def call_noalloc(L, t, w, out):
+    """fa_bwd_noalloc through the C ABI with raw device pointers."""
+    q, k, v, o, do, lse, kv = t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["kv_len"]
+    return L.fa_bwd_noalloc(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+        ctypes.c_void_p(do.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+        ctypes.c_void_p(out["dq"].data_ptr()), ctypes.c_void_p(out["dk"].data_ptr()),
+        ctypes.c_void_p(out["dv"].data_ptr()), w.B, w.H, w.N, w.d, ctypes.c_float(w.scale),
+        int(w.causal), None if kv is None else ctypes.c_void_p(kv.data_ptr()),
+        fa.FA_BF16 if w.dtype == torch.bfloat16 else fa.FA_FP16,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_noalloc_matches_workspace_entry_point_on_two_calls(w):
+    L = fa.lib()
+    dev = torch.device("cuda", 0)
+    inp = W.make_inputs(w, seed=77)
+    t = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
+    t["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
+    t["o"], t["lse"] = fa.forward(t["q"], t["k"], t["v"], scale=w.scale, causal=w.causal,
+                                  kv_len=t["kv_len"])
+    ref = dict(zip(("dq", "dk", "dv"),
+                   fa.backward(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], scale=w.scale,
+                               causal=w.causal, kv_len=t["kv_len"])))
+    torch.cuda.synchronize()
+    for call in range(2):
+        # start from garbage so that stale outputs cannot pass
+        out = {n: torch.full_like(t["q"], float("nan")) for n in ("dq", "dk", "dv")}
+        assert call_noalloc(L, t, w, out) == fa.FA_OK
+        torch.cuda.synchronize()
+        assert fa.fa_get_device_status() == fa.FA_OK
+        for n in ("dq", "dk", "dv"):
+            err = rel_l2(out[n].double().cpu().numpy(), ref[n].double().cpu().numpy())
+            assert err <= GRAD_REL_L2, (call, n, err)
+
+
+def test_noalloc_refuses_problems_beyond_its_scratch():
+    L = fa.lib()
+    dev = torch.device("cuda", 0)
+    # workspace for B1 H1 N=129152 d=128 exceeds the static 64 MiB
+    w = W.custom("too-big", B=1, H=1, N=129152, d=128, dtype=torch.bfloat16)
+    assert L.fa_bwd_workspace_bytes(1, 1, w.N, w.d) > fa.FA_NOALLOC_SCRATCH_BYTES
+    x = torch.zeros(1, 1, w.N, w.d, dtype=w.dtype, device=dev)
+    lse = torch.zeros(1, 1, w.N, device=dev)
+    t = {"q": x, "k": x, "v": x, "o": x, "do": x, "lse": lse, "kv_len": None}
+    out = {n: torch.full_like(x, 7.0) for n in ("dq", "dk", "dv")}
+    assert call_noalloc(L, t, w, out) == fa.FA_ERR_SCRATCH_LIMIT
+    torch.cuda.synchronize()
+    assert all(bool(torch.all(out[n] == 7.0)) for n in ("dq", "dk", "dv"))  # nothing ran
+    assert fa.fa_strerror(fa.FA_ERR_SCRATCH_LIMIT).startswith("problem needs more scratch")
