@@ -137,6 +137,9 @@ struct BwdCfg {
     static constexpr int HALF = 128 * 128;    // one 128-byte column block of a tile
     static constexpr int HALVES = D / 64;
     static constexpr bool DQ_TMA = (D == 64);  // dQ drain by TMA reduce (else red.v4)
+    // d = 64: P^T gets its own TMEM columns, so S_{i+1} can overwrite S_i as soon as it
+    // has been read.  d = 128: TMEM is full; P^T overwrites S^T and S_{i+1} waits for dV_i.
+    static constexpr bool P_OWN = (D == 64);
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + TILE;
     static constexpr int OFF_Q = OFF_V + TILE;       // 2 stages
@@ -151,13 +154,21 @@ struct BwdCfg {
     // d = 128 uses all 227 KB: no room for alignment slack; the kernel checks instead.
     static constexpr int SLACK = (USED + 1024 <= 232448) ? 1024 : 0;
     static constexpr int SMEM = USED + SLACK;
-    static constexpr int THREADS = 320;
+    // warps 0..7: P / dS (lane quarter w % 4, query half w / 4); 8: TMA; 9: MMA;
+    // 10..13: dQ drain (lane quarters 2, 3, 0, 1).
+    static constexpr int THREADS = 448;
+    static constexpr int W_TMA = 8, W_MMA = 9, W_DQ0 = 10;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0;
     static constexpr uint32_t COL_DP = 128;
     static constexpr uint32_t COL_DV = 256;
     static constexpr uint32_t COL_DK = 256 + D;
     static constexpr uint32_t COL_DQ = (D == 64) ? 384 : 128;  // d = 128: aliases dP^T
+    static constexpr uint32_t COL_P = P_OWN ? 448 : COL_S;
+    // Column of the 16-bit pairs of queries 64h..64h+63 inside the P^T / dS^T areas:
+    // each query half is written over columns its own warp has already read.
+    static constexpr uint32_t P_HALF_STRIDE = P_OWN ? 32 : 64;
+    static constexpr uint32_t DS_HALF_STRIDE = 64;
 };
 
 struct BwdBars {
@@ -165,12 +176,13 @@ struct BwdBars {
     uint64_t q_full[2];
     uint64_t do_full[2];
     uint64_t stage_empty[2];
-    uint64_t s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_empty, dkv_full;
+    uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
+        dkv_full;
     uint32_t tmem_base;
 };
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
               const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -208,7 +220,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int q_begin = p.causal ? kt : 0;
     const int n = (kt * 128 < L) ? (p.num_tiles - q_begin) : 0;  // query tiles visited
 
-    if (threadIdx.x == 128) {
+    if (warp == C::W_TMA && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -223,22 +235,24 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(&bars->stage_empty[i], 1);
         }
         mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_free, 256);
         mbar_init(&bars->dp_full, 1);
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->ds_full, 128);
+        mbar_init(&bars->p_full, 256);
+        mbar_init(&bars->p_free, 1);
+        mbar_init(&bars->ds_full, 256);
         mbar_init(&bars->ds_empty, 1);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 128);
         mbar_init(&bars->dkv_full, 1);
         fence_mbar_init();
     }
-    if (warp == 5) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    if (warp == C::W_MMA) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 4) {
+    if (warp == C::W_TMA) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0 && n > 0) {
             mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
@@ -263,7 +277,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 bulk_load(sDv + s * 128, p.dvec + vec_off, 512, &bars->do_full[s]);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::W_MMA) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0 && n > 0) {
             constexpr uint32_t kIdescSq = idesc_f16(BF16, false, false, 128, 128);  // S^T, dP^T
@@ -281,11 +295,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                            smem_desc_sw128(b_base + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
                 }
             };
-            // D[128 x D] (+)= A_tmem[128 x 128] * B[128 rows][D] (MN-major B).
-            auto mma_tmem_a = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool acc) {
+            // D[128 x D] (+)= A_tmem[128 x 128] * B[128 rows][D] (MN-major B).  The A pairs
+            // of queries 64..127 start `half_stride` columns after those of queries 0..63.
+            auto mma_tmem_a = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t half_stride,
+                                  uint32_t b_base, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(d_tmem, a_tmem + kk * 8,
+                    mma_ts(d_tmem, a_tmem + (kk >> 2) * half_stride + (kk & 3) * 8,
                            smem_desc_sw128(b_base + kk * 2048, C::HALF, 1024), kIdescTs,
                            (acc || kk > 0) ? 1u : 0u);
             };
@@ -304,10 +320,22 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             for (int i = 0; ok && i < n; ++i) {
                 const int s = i & 1;
+                if (C::P_OWN && i + 1 < n) {
+                    // S_{i+1} overwrites S_i as soon as every P/dS warp has read it.
+                    const int s1 = (i + 1) & 1;
+                    if (!mbar_wait(&bars->s_free, i & 1)) break;
+                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
+                    tc_fence_after();
+                    mma_square(tmem + C::COL_S, k_addr, q_addr + s1 * C::TILE);
+                    mma_commit(&bars->s_full);
+                }
                 if (!mbar_wait(&bars->p_full, i & 1)) break;
                 tc_fence_after();
-                mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_S, do_addr + s * C::TILE, i > 0);
-                if (i + 1 < n) {
+                mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE, do_addr + s * C::TILE,
+                           i > 0);
+                mma_commit(&bars->p_free);
+                if (!C::P_OWN && i + 1 < n) {
+                    // P^T_i lives in the S^T columns: S_{i+1} follows dV_i.
                     const int s1 = (i + 1) & 1;
                     if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
                     tc_fence_after();
@@ -316,7 +344,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 if (!mbar_wait(&bars->ds_full, i & 1)) break;
                 tc_fence_after();
-                mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, q_addr + s * C::TILE, i > 0);
+                mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
+                           q_addr + s * C::TILE, i > 0);
                 if (D == 64 && i > 0) {
                     if (!mbar_wait(&bars->dq_empty, (i - 1) & 1)) break;
                     tc_fence_after();
@@ -343,40 +372,32 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             mma_commit(&bars->dkv_full);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= C::W_DQ0) {
         // ------------------------------ dQ drain ----------------------------------
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;  // query row in the tile = TMEM lane
-        const int gt = threadIdx.x - 192;   // 0..127 inside this warpgroup
+        const int r = quarter * 32 + lane;          // query row in the tile = TMEM lane
+        const int gt = threadIdx.x - C::W_DQ0 * 32;  // 0..127 inside this warpgroup
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         for (int i = 0; i < n; ++i) {
             const int qi = q_begin + i;
             if (!mbar_wait(&bars->dq_full, i & 1)) break;
             tc_fence_after();
-            float v[D];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t w[32];
-                tmem_ld32(tmem + lane_base + C::COL_DQ + c * 32, w);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) v[c * 32 + k] = __uint_as_float(w[k]);
-            }
-            tc_fence_before();
-            mbar_arrive(&bars->dq_empty);
             if constexpr (C::DQ_TMA) {
                 if (gt == 0) bulk_wait_group_read<0>();
                 named_bar_sync(2, 128);
                 // D/32 boxes of [128 rows][32 fp32], 16-byte chunks swizzled by row % 8.
 #pragma unroll
                 for (int bx = 0; bx < D / 32; ++bx) {
+                    uint32_t w[32];
+                    tmem_ld32(tmem + lane_base + C::COL_DQ + bx * 32, w);
                     uint8_t *rowp = sDQ + bx * 16384 + r * 128;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float *x = v + bx * 32 + c * 4;
-                        *reinterpret_cast<float4 *>(rowp + ((c ^ (r & 7)) << 4)) =
-                            make_float4(x[0], x[1], x[2], x[3]);
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(rowp + ((c ^ (r & 7)) << 4)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
                 }
+                tc_fence_before();
+                mbar_arrive(&bars->dq_empty);
                 fence_proxy_async_smem();
                 named_bar_sync(2, 128);
                 if (gt == 0) {
@@ -387,11 +408,21 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
             } else {
                 const int row = qi * 128 + r;
-                if (row < p.N) {
-                    float *dst = p.dq_acc + ((size_t)bh * p.N + row) * D;
+                float *dst = p.dq_acc + ((size_t)bh * p.N + (row < p.N ? row : 0)) * D;
 #pragma unroll
-                    for (int c = 0; c < D; c += 4) red_add_v4(dst + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tmem + lane_base + C::COL_DQ + c * 32, w);
+                    if (row < p.N) {
+#pragma unroll
+                        for (int k = 0; k < 32; k += 4)
+                            red_add_v4(dst + c * 32 + k, __uint_as_float(w[k]),
+                                       __uint_as_float(w[k + 1]), __uint_as_float(w[k + 2]),
+                                       __uint_as_float(w[k + 3]));
+                    }
                 }
+                tc_fence_before();
+                mbar_arrive(&bars->dq_empty);
             }
         }
         if constexpr (C::DQ_TMA) {
@@ -399,10 +430,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
     } else {
         // ------------------------------ P / dS warps ------------------------------
-        const int t = threadIdx.x;  // key row in the tile = TMEM lane
+        const int quarter = warp & 3;
+        const int h = warp >> 2;             // query half: columns 64h .. 64h + 63
+        const int t = quarter * 32 + lane;   // key row in the tile = TMEM lane
         const int key = kt * 128 + t;
         const bool key_ok = key < L;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
         for (int i = 0; i < n; ++i) {
@@ -413,41 +446,45 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 break;
             }
             tc_fence_after();
-            // P^T row, kept as packed 16-bit pairs (exactly what the dV MMA consumes);
-            // dS below uses the same rounded values.
-            uint32_t Pw[64];
-            const float *lse2 = sLSE + s * 128;
-            const bool diag = p.causal && (qi == kt);
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t w[32];
-                tmem_ld32(tmem + lane_base + C::COL_S + cc * 32, w);
-#pragma unroll
-                for (int k = 0; k < 32; k += 4) {
-                    const int c = cc * 32 + k;
-                    const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + c);
-                    float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
-                    float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
-                    float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
-                    float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
-                    // masked: keys past the valid length, queries before the key (causal)
-                    if (!key_ok || (diag && c < t)) p0 = 0.f;
-                    if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
-                    if (!key_ok || (diag && c + 2 < t)) p2 = 0.f;
-                    if (!key_ok || (diag && c + 3 < t)) p3 = 0.f;
-                    Pw[c >> 1] = pack2<BF16>(p0, p1);
-                    Pw[(c >> 1) + 1] = pack2<BF16>(p2, p3);
-                }
-            }
+            // P^T for queries 64h .. 64h + 63 of this key row, packed in 16-bit pairs
+            // (exactly what the dV MMA consumes; dS below uses the same rounded values).
+            uint32_t Pw[32];
             {
-                uint32_t w[32];
+                uint32_t w0[32], w1[32];
+                tmem_ld32(tmem + lane_base + C::COL_S + h * 64, w0);
+                tmem_ld32(tmem + lane_base + C::COL_S + h * 64 + 32, w1);
+                if (C::P_OWN) {
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free);  // S^T may now be overwritten by S_{i+1}
+                }
+                const float *lse2 = sLSE + s * 128 + h * 64;
+                const bool diag = p.causal && (qi == kt);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) w[k] = Pw[h * 32 + k];
-                    tmem_st32(tmem + lane_base + C::COL_S + h * 32, w);
+                    for (int k = 0; k < 32; k += 4) {
+                        const uint32_t *w = cc == 0 ? w0 : w1;
+                        const int c = h * 64 + cc * 32 + k;  // query column in the tile
+                        const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + cc * 32 + k);
+                        float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
+                        float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
+                        float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
+                        float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
+                        // masked: keys past the valid length, queries before the key (causal)
+                        if (!key_ok || (diag && c < t)) p0 = 0.f;
+                        if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
+                        if (!key_ok || (diag && c + 2 < t)) p2 = 0.f;
+                        if (!key_ok || (diag && c + 3 < t)) p3 = 0.f;
+                        Pw[cc * 16 + (k >> 1)] = pack2<BF16>(p0, p1);
+                        Pw[cc * 16 + (k >> 1) + 1] = pack2<BF16>(p2, p3);
+                    }
                 }
             }
+            if (C::P_OWN && i > 0 && !mbar_wait(&bars->p_free, (i - 1) & 1)) {  // dV_{i-1} read P
+                ok = false;
+                break;
+            }
+            tmem_st32(tmem + lane_base + C::COL_P + h * C::P_HALF_STRIDE, Pw);
             tc_fence_before();
             mbar_arrive(&bars->p_full);
 
@@ -457,29 +494,29 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 break;
             }
             tc_fence_after();
-            const float *dv = sDv + s * 128;
+            const float *dv = sDv + s * 128 + h * 64;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t w[32];
-                tmem_ld32(tmem + lane_base + C::COL_DP + cc * 32, w);
+                tmem_ld32(tmem + lane_base + C::COL_DP + h * 64 + cc * 32, w);
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const int c = cc * 32 + k;
-                    const float2 d2 = *reinterpret_cast<const float2 *>(dv + c);
-                    const float2 pp = unpack2<BF16>(Pw[c >> 1]);
+                    const float2 d2 = *reinterpret_cast<const float2 *>(dv + cc * 32 + k);
+                    const float2 pp = unpack2<BF16>(Pw[cc * 16 + (k >> 1)]);
                     const float ds0 = pp.x * (__uint_as_float(w[k]) - d2.x);
                     const float ds1 = pp.y * (__uint_as_float(w[k + 1]) - d2.y);
                     pk[k >> 1] = pack2<BF16>(ds0, ds1);
                 }
-                // dS^T row -> TMEM (columns already read), A operand of dK += dS^T Q.
-                tmem_st16(tmem + lane_base + C::COL_DP + cc * 16, pk);
+                // dS^T pairs -> TMEM, over dP^T columns this warp has just read; A operand
+                // of dK += dS^T Q.
+                tmem_st16(tmem + lane_base + C::COL_DP + h * C::DS_HALF_STRIDE + cc * 16, pk);
                 // dS -> shared memory as the MN-major A operand of dQ = dS K:
-                // [query block (64)][key row t][64 queries], 128-byte swizzle.
-                uint8_t *rowp = sdS + (cc >> 1) * 16384 + t * 128;
+                // [query block h (64 queries)][key row t][128 bytes], 128-byte swizzle.
+                uint8_t *rowp = sdS + h * 16384 + t * 128;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const int chunk = (cc & 1) * 4 + q4;
+                    const int chunk = cc * 4 + q4;
                     *reinterpret_cast<uint4 *>(rowp + ((chunk ^ (t & 7)) << 4)) =
                         make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
                 }
@@ -494,41 +531,44 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             ok = mbar_wait(&bars->dkv_full, 0);
             tc_fence_after();
         }
-        // Staging: the first Q / dO stage buffers are free once every MMA is done.
+        // Staging: the first Q / dO stage buffers are free once every MMA is done.  Each
+        // warp converts its lane quarter's D/2 columns of dV and dK.
         uint8_t *stage_v = sQ;
         uint8_t *stage_k = sdO;
+        constexpr int HCOLS = D / 2;  // columns of this warp's half
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
-            const uint32_t col = which == 0 ? C::COL_DV : C::COL_DK;
+            const uint32_t col = (which == 0 ? C::COL_DV : C::COL_DK) + h * HCOLS;
             const float mul = which == 0 ? 1.f : p.scale;
             uint8_t *stage = which == 0 ? stage_v : stage_k;
 #pragma unroll
-            for (int hf = 0; hf < C::HALVES; ++hf) {
-                uint32_t wv[32];
+            for (int c32 = 0; c32 < HCOLS / 32; ++c32) {
+                uint32_t w[32];
+                if (n > 0) {
+                    tmem_ld32(tmem + lane_base + col + c32 * 32, w);
+                } else {
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t w[32];
-                    if (n > 0) {
-                        tmem_ld32(tmem + lane_base + col + hf * 64 + h2 * 32, w);
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) w[k] = 0u;
-                    }
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        wv[h2 * 16 + k] = pack2<BF16>(__uint_as_float(w[2 * k]) * mul,
-                                                      __uint_as_float(w[2 * k + 1]) * mul);
+                    for (int k = 0; k < 32; ++k) w[k] = 0u;
                 }
-                uint8_t *rowp = stage + hf * C::HALF + t * 128;
+                uint32_t wv[16];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(rowp + ((c ^ (t & 7)) << 4)) =
+                for (int k = 0; k < 16; ++k)
+                    wv[k] = pack2<BF16>(__uint_as_float(w[2 * k]) * mul,
+                                        __uint_as_float(w[2 * k + 1]) * mul);
+                // element e = h * HCOLS + c32 * 32 .. + 31 of row t: 128-byte block e / 64,
+                // 16-byte chunks (e % 64) / 8 .. + 3
+                const int e0 = h * HCOLS + c32 * 32;
+                uint8_t *rowp = stage + (e0 >> 6) * C::HALF + t * 128;
+                const int ch0 = (e0 & 63) >> 3;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4 *>(rowp + (((ch0 + c) ^ (t & 7)) << 4)) =
                         make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
             }
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (t == 0) {
+        named_bar_sync(1, 256);
+        if (threadIdx.x == 0) {
             for (int hf = 0; hf < C::HALVES; ++hf) {
                 tma_store_3d(&tmdV, stage_v + hf * C::HALF, hf * 64, kt * 128, bh);
                 tma_store_3d(&tmdK, stage_k + hf * C::HALF, hf * 64, kt * 128, bh);
@@ -541,7 +581,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == C::W_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fa

@@ -10,9 +10,10 @@
 // B200 mapping (one CTA = one 128-row query tile of one (batch, head)):
 //   warp 4      TMA producer: Q once, then K_j / V_j into an NS-stage shared-memory ring
 //               (128-byte swizzle, mbarrier transaction counts).
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM (double-buffered, so the
-//               next block's scores are computed while softmax works on this one), then
-//               O += P_j V_j with P_j read straight from TMEM.
+//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM, then O += P_j V_j with
+//               P_j read straight from TMEM.  d = 128: two score buffers, so the next
+//               block's scores are computed while softmax works on this one.  d = 64: one
+//               score buffer and two CTAs per SM, so the other CTA fills the gaps.
 //   warps 0..3  softmax, one query row per thread (TMEM lane = row): load S_j, mask on
 //               diagonal / tail blocks only, row max, p = 2^(s*scale*log2e - m) with the
 //               MUFU ex2, row sum, P_j written back into TMEM as 16-bit pairs over S_j.
@@ -54,7 +55,13 @@ struct FwdCfg {
     static constexpr int HALVES = D / 64;               // 128-byte column blocks per row
     static constexpr int TILE = BM * D * 2;             // bytes of one Q / K / V tile
     static constexpr int HALF = BM * 128;               // bytes of one column block
-    static constexpr int NS = (D == 64) ? 4 : 2;        // K/V ring depth
+    // d = 64: one score buffer in TMEM (256 columns) and a 2-stage ring (83 KB), so two
+    // CTAs share an SM and one CTA's softmax overlaps the other's MMAs and epilogue.
+    // d = 128: the CTA owns the SM, with two score buffers so that S_{j+1} is computed
+    // while softmax works on S_j.
+    static constexpr int SBUF = (D == 64) ? 1 : 2;      // score buffers in TMEM
+    static constexpr int CTAS_PER_SM = (D == 64) ? 2 : 1;
+    static constexpr int NS = 2;                        // K/V ring depth
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + TILE;
     static constexpr int OFF_V = OFF_K + NS * TILE;
@@ -62,9 +69,9 @@ struct FwdCfg {
     static constexpr int OFF_BAR = OFF_ONES + 2048;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;   // + barriers + alignment slack
     static constexpr int THREADS = 192;
-    static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_O = 256;              // S0 at 0, S1 at 128, O at 256
-    static constexpr uint32_t COL_SUM = 256 + D;        // 16 columns: row sums of 16-bit P
+    static constexpr uint32_t TMEM_COLS = (SBUF == 1) ? 256 : 512;
+    static constexpr uint32_t COL_O = SBUF * 128;       // S buffers first, then O
+    static constexpr uint32_t COL_SUM = COL_O + D;      // 16 columns: row sums of 16-bit P
 };
 
 struct FwdBars {
@@ -79,7 +86,7 @@ struct FwdBars {
 };
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
               const FwdParams p) {
@@ -175,7 +182,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const int s = j % C::NS;
                 if (!mbar_wait(&bars->k_full[s], (j / C::NS) & 1)) return false;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 128);
+                const uint32_t d_tmem = tmem + (uint32_t)((j % C::SBUF) * 128);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * C::HALF + (kk & 3) * 32);
@@ -183,17 +190,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const uint64_t bd = smem_desc_sw128(k_addr + s * C::TILE + off, 16, 1024);
                     mma_ss(d_tmem, a, bd, kIdescS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full[j & 1]);
+                mma_commit(&bars->s_full[j % C::SBUF]);
                 return true;
             };
             if (ok) ok = issue_s(0);
             for (int j = 0; ok && j < T; ++j) {
-                if (j + 1 < T && !issue_s(j + 1)) break;
+                // With two score buffers S_{j+1} goes ahead of P_j V_j; with one it has to
+                // follow it, since P_j lives in the buffer S_{j+1} overwrites.
+                if (C::SBUF == 2 && j + 1 < T && !issue_s(j + 1)) break;
                 const int s = j % C::NS;
-                if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1)) break;
+                if (!mbar_wait(&bars->p_full[j % C::SBUF], (j / C::SBUF) & 1)) break;
                 if (!mbar_wait(&bars->v_full[s], (j / C::NS) & 1)) break;
                 tc_fence_after();
-                const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 128);
+                const uint32_t p_tmem = tmem + (uint32_t)((j % C::SBUF) * 128);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
                     const uint64_t bd =
@@ -207,6 +216,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                            (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bars->kv_empty[s]);
                 mma_commit(&bars->o_full);
+                if (C::SBUF == 1 && j + 1 < T && !issue_s(j + 1)) break;
             }
         }
     } else {
@@ -219,9 +229,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float l = 0.f;        // running normaliser
         bool ok = true;
         for (int j = 0; j < T; ++j) {
-            if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars->s_full[j % C::SBUF], (j / C::SBUF) & 1)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sb = tmem + lane_base + (uint32_t)((j & 1) * 128);
+            const uint32_t sb = tmem + lane_base + (uint32_t)((j % C::SBUF) * 128);
             float s[128];
             {
                 uint32_t r[32];
@@ -305,7 +315,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->p_full[j & 1]);
+            mbar_arrive(&bars->p_full[j % C::SBUF]);
         }
 
         // ------------------------------ epilogue ------------------------------
