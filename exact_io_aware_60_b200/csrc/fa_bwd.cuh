@@ -283,39 +283,46 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             constexpr uint32_t kIdescSq = idesc_f16(BF16, false, false, 128, 128);  // S^T, dP^T
             constexpr uint32_t kIdescTs = idesc_f16(BF16, false, true, 128, D);     // dV, dK
             constexpr uint32_t kIdescDq = idesc_f16(BF16, true, true, 128, D);      // dQ
-            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-            const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO);
-            const uint32_t ds_addr = smem_u32(sdS);
+            // Descriptors are built once; per k-step and per stage only the 16-byte start
+            // address field changes, by compile-time offsets.
+            const uint64_t k_kmaj = smem_desc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t v_kmaj = smem_desc_sw128(smem_u32(sV), 16, 1024);
+            const uint64_t q_kmaj = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t do_kmaj = smem_desc_sw128(smem_u32(sdO), 16, 1024);
+            const uint64_t q_mn = smem_desc_sw128(smem_u32(sQ), C::HALF, 1024);
+            const uint64_t do_mn = smem_desc_sw128(smem_u32(sdO), C::HALF, 1024);
+            const uint64_t k_mn = smem_desc_sw128(smem_u32(sK), C::HALF, 1024);
+            const uint64_t ds_mn = smem_desc_sw128(smem_u32(sdS), 16384, 1024);
             // X^T = A B^T with A, B both [128 rows][D] K-major tiles.
-            auto mma_square = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+            auto mma_square = [&](uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * C::HALF + (kk & 3) * 32);
-                    mma_ss(d_tmem, smem_desc_sw128(a_base + off, 16, 1024),
-                           smem_desc_sw128(b_base + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
+                    mma_ss(d_tmem, a_desc + off, b_desc + off, kIdescSq, kk > 0 ? 1u : 0u);
                 }
             };
             // D[128 x D] (+)= A_tmem[128 x 128] * B[128 rows][D] (MN-major B).  The A pairs
             // of queries 64..127 start `half_stride` columns after those of queries 0..63.
             auto mma_tmem_a = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t half_stride,
-                                  uint32_t b_base, bool acc) {
+                                  uint64_t b_desc, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(d_tmem, a_tmem + (kk >> 2) * half_stride + (kk & 3) * 8,
-                           smem_desc_sw128(b_base + kk * 2048, C::HALF, 1024), kIdescTs,
+                           b_desc + (uint64_t)(kk * 2048 >> 4), kIdescTs,
                            (acc || kk > 0) ? 1u : 0u);
             };
+            auto stage_off = [](int st) { return (uint64_t)((st * C::TILE) >> 4); };
             bool ok = mbar_wait(&bars->kv_full, 0);
             ok = ok && mbar_wait(&bars->q_full[0], 0);
             tc_fence_after();
             if (ok) {
-                mma_square(tmem + C::COL_S, k_addr, q_addr);
+                mma_square(tmem + C::COL_S, k_kmaj, q_kmaj);
                 mma_commit(&bars->s_full);
                 ok = mbar_wait(&bars->do_full[0], 0);
                 tc_fence_after();
             }
             if (ok) {
-                mma_square(tmem + C::COL_DP, v_addr, do_addr);
+                mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj);
                 mma_commit(&bars->dp_full);
             }
             for (int i = 0; ok && i < n; ++i) {
@@ -326,12 +333,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if (!mbar_wait(&bars->s_free, i & 1)) break;
                     if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
                     tc_fence_after();
-                    mma_square(tmem + C::COL_S, k_addr, q_addr + s1 * C::TILE);
+                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
                     mma_commit(&bars->s_full);
                 }
                 if (!mbar_wait(&bars->p_full, i & 1)) break;
                 tc_fence_after();
-                mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE, do_addr + s * C::TILE,
+                mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE, do_mn + stage_off(s),
                            i > 0);
                 mma_commit(&bars->p_free);
                 if (!C::P_OWN && i + 1 < n) {
@@ -339,22 +346,21 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const int s1 = (i + 1) & 1;
                     if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
                     tc_fence_after();
-                    mma_square(tmem + C::COL_S, k_addr, q_addr + s1 * C::TILE);
+                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
                     mma_commit(&bars->s_full);
                 }
                 if (!mbar_wait(&bars->ds_full, i & 1)) break;
                 tc_fence_after();
                 mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
-                           q_addr + s * C::TILE, i > 0);
+                           q_mn + stage_off(s), i > 0);
                 if (D == 64 && i > 0) {
                     if (!mbar_wait(&bars->dq_empty, (i - 1) & 1)) break;
                     tc_fence_after();
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + C::COL_DQ, smem_desc_sw128(ds_addr + kk * 2048, 16384, 1024),
-                           smem_desc_sw128(k_addr + kk * 2048, C::HALF, 1024), kIdescDq,
-                           kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
+                           k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
                 mma_commit(&bars->ds_empty);
                 mma_commit(&bars->stage_empty[s]);
@@ -366,7 +372,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                     if (!mbar_wait(&bars->do_full[s1], ((i + 1) >> 1) & 1)) break;
                     tc_fence_after();
-                    mma_square(tmem + C::COL_DP, v_addr, do_addr + s1 * C::TILE);
+                    mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
                     mma_commit(&bars->dp_full);
                 }
             }

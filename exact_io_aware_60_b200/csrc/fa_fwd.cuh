@@ -11,21 +11,30 @@
 //   warp 4      TMA producer: Q once, then K_j / V_j into an NS-stage shared-memory ring
 //               (128-byte swizzle, mbarrier transaction counts).
 //   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM, then O += P_j V_j with
-//               P_j read straight from TMEM.  d = 128: two score buffers, so the next
-//               block's scores are computed while softmax works on this one.  d = 64: one
-//               score buffer and two CTAs per SM, so the other CTA fills the gaps.
+//               P_j read straight from TMEM.
 //   warps 0..3  softmax, one query row per thread (TMEM lane = row): load S_j, mask on
 //               diagonal / tail blocks only, row max, p = 2^(s*scale*log2e - m) with the
-//               MUFU ex2, row sum, P_j written back into TMEM as 16-bit pairs over S_j.
+//               MUFU ex2, row sum, P_j written back into TMEM as 16-bit pairs.
 //               The output rescale is lazy: m only moves when the row max grows by more
 //               than 2^8, which leaves the result exact because O and l always share the
 //               same m.  Epilogue: O / l' -> 16-bit, staged swizzled in shared memory and
 //               written with one TMA store; LSE = ln2 * (m + log2 l).
 //   Normaliser: the tensor core multiplies V by P rounded to 16 bits, so the output is
-//   divided by l' = sum of exactly those rounded values, produced by one more small MMA
-//   (P times a tile of ones) into 16 spare TMEM columns.  The weights applied to the rows
-//   of V then sum to one exactly, which removes the bias a fp32 l would leave when one
-//   key dominates a row.  LSE keeps the fp32 sum l of the unrounded values.
+//   divided by l' = sum of exactly those rounded values, produced by the same PV MMA
+//   (its B operand carries 16 extra columns of ones after V) in 16 extra TMEM columns.
+//   The weights applied to the rows of V then sum to one exactly, which removes the bias
+//   a fp32 l would leave when one key dominates a row.  LSE keeps the fp32 sum l of the
+//   unrounded values.
+//
+// Two shapes of the same kernel:
+//   d = 64  : 64-key blocks; TMEM holds S (64 columns), P (32), O and the sums (80): 176
+//             of 256 columns, so two CTAs share an SM.  P has its own columns, so S_{j+1}
+//             is computed as soon as the softmax has read S_j, while it works on P_j.
+//   d = 128 : 128-key blocks; the CTA owns the SM's 512 columns: two score buffers (P_j is
+//             written over S_j), so S_{j+1} is computed while softmax works on S_j.
+// A tcgen05.mma instruction costs at least ~45 cycles whatever its N, so small MMAs are
+// merged where possible (the row sums ride on the PV instruction).
+//
 // The loop order is query-block outer (each CTA writes its O rows once) instead of the
 // key-block-outer order of the original algorithm; the result is the same up to
 // floating-point ordering.
@@ -51,32 +60,42 @@ struct FwdParams {
 template <int D>
 struct FwdCfg {
     static constexpr int BM = 128;                      // query rows per tile
-    static constexpr int BN = 128;                      // keys per block
+    static constexpr int BN = (D == 64) ? 64 : 128;     // keys per block
     static constexpr int HALVES = D / 64;               // 128-byte column blocks per row
-    static constexpr int TILE = BM * D * 2;             // bytes of one Q / K / V tile
-    static constexpr int HALF = BM * 128;               // bytes of one column block
-    // d = 64: one score buffer in TMEM (256 columns) and a 2-stage ring (83 KB), so two
-    // CTAs share an SM and one CTA's softmax overlaps the other's MMAs and epilogue.
-    // d = 128: the CTA owns the SM, with two score buffers so that S_{j+1} is computed
-    // while softmax works on S_j.
+    static constexpr int QTILE = BM * D * 2;            // bytes of the Q tile
+    static constexpr int QHALF = BM * 128;              // one column block of Q
+    static constexpr int KTILE = BN * D * 2;            // bytes of one K or V block
+    static constexpr int KHALF = BN * 128;              // one column block of K or V
+    static constexpr bool P_OWN = (D == 64);            // P in its own TMEM columns
     static constexpr int SBUF = (D == 64) ? 1 : 2;      // score buffers in TMEM
     static constexpr int CTAS_PER_SM = (D == 64) ? 2 : 1;
-    static constexpr int NS = 2;                        // K/V ring depth
+    static constexpr int NS = (D == 64) ? 4 : 2;        // K/V ring depth
+    // Each V stage is followed by a block of 16-bit ones, one 64-column block past the
+    // tile: the PV MMA reads it as B columns D..D+15 and so also produces the row sums
+    // of P (one N = D + 16 instruction instead of a second, equally costly N = 16 one).
+    static constexpr int VSTAGE = (HALVES + 1) * KHALF;  // V block + its ones block
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE;
-    static constexpr int OFF_V = OFF_K + NS * TILE;
-    static constexpr int OFF_ONES = OFF_V + NS * TILE;   // 2 KB of 16-bit ones
-    static constexpr int OFF_BAR = OFF_ONES + 2048;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;   // + barriers + alignment slack
+    static constexpr int OFF_K = OFF_Q + QTILE;
+    static constexpr int OFF_V = OFF_K + NS * KTILE;
+    static constexpr int OFF_BAR = OFF_V + NS * VSTAGE;
+    static constexpr int USED = OFF_BAR + 256;
+    // Two CTAs per SM leave no room for an alignment pad at d = 64: the kernel checks
+    // that the dynamic shared-memory base is 1024-byte aligned instead.
+    static constexpr int SLACK = (CTAS_PER_SM == 1) ? 1024 : 0;
+    static constexpr int SMEM = USED + SLACK;
     static constexpr int THREADS = 192;
-    static constexpr uint32_t TMEM_COLS = (SBUF == 1) ? 256 : 512;
-    static constexpr uint32_t COL_O = SBUF * 128;       // S buffers first, then O
+    static constexpr uint32_t TMEM_COLS = (CTAS_PER_SM == 2) ? 256 : 512;
+    static constexpr uint32_t COL_P = SBUF * BN;        // d = 64 only: 32 columns
+    static constexpr uint32_t COL_O = P_OWN ? COL_P + BN / 2 : SBUF * BN;
     static constexpr uint32_t COL_SUM = COL_O + D;      // 16 columns: row sums of 16-bit P
+    static constexpr int PV_N = D + 16;                 // O and the row sums in one MMA
+    static_assert(COL_SUM + 16 <= TMEM_COLS, "TMEM budget");
 };
 
 struct FwdBars {
     uint64_t q_full;
     uint64_t s_full[2];
+    uint64_t s_read;
     uint64_t p_full[2];
     uint64_t o_full;
     uint64_t k_full[4];
@@ -91,8 +110,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
               const FwdParams p) {
     using C = FwdCfg<D>;
+    constexpr int BN = C::BN;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad > (uint32_t)C::SLACK) {  // cannot happen with a 1024-aligned dynamic base
+        if (threadIdx.x == 0) atomicExch(&g_status, 5);
+        return;
+    }
     uint8_t *smem = smem_raw + pad;
     uint8_t *sQ = smem + C::OFF_Q;
     uint8_t *sK = smem + C::OFF_K;
@@ -114,7 +138,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     int kv_end = L;
     if (p.causal) kv_end = min(kv_end, (qt + 1) * C::BM);
-    const int T = (kv_end + C::BN - 1) / C::BN;  // key blocks this tile visits
+    const int T = (kv_end + BN - 1) / BN;  // key blocks this tile visits
 
     if (threadIdx.x == 128) {
         tma_prefetch_desc(&tmQ);
@@ -126,6 +150,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], 128);
         }
+        mbar_init(&bars->s_read, 128);
         mbar_init(&bars->o_full, 1);
         for (int i = 0; i < C::NS; ++i) {
             mbar_init(&bars->k_full[i], 1);
@@ -135,10 +160,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         fence_mbar_init();
     }
     if (warp == 4) {
-        // 16-bit ones: B operand of the row-sum MMA (layout-agnostic: every element is 1)
+        // 16-bit ones after every V stage (layout-agnostic: every element is 1)
         const uint32_t one2 = BF16 ? 0x3F803F80u : 0x3C003C00u;
-        uint32_t *ones = reinterpret_cast<uint32_t *>(smem + C::OFF_ONES);
-        for (int i = lane; i < 512; i += 32) ones[i] = one2;
+        for (int st = 0; st < C::NS; ++st) {
+            uint4 *ones = reinterpret_cast<uint4 *>(sV + st * C::VSTAGE + C::HALVES * C::KHALF);
+            for (int i = lane; i < C::KHALF / 16; i += 32) ones[i] = make_uint4(one2, one2, one2, one2);
+        }
         fence_proxy_async_smem();
     }
     if (warp == 5) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
@@ -150,73 +177,72 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (warp == 4) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0 && T > 0) {
-            mbar_arrive_expect_tx(&bars->q_full, C::TILE);
+            mbar_arrive_expect_tx(&bars->q_full, C::QTILE);
             for (int hf = 0; hf < C::HALVES; ++hf)
-                tma_load_3d(sQ + hf * C::HALF, &tmQ, &bars->q_full, hf * 64, qt * C::BM, bh);
+                tma_load_3d(sQ + hf * C::QHALF, &tmQ, &bars->q_full, hf * 64, qt * C::BM, bh);
             for (int j = 0; j < T; ++j) {
                 const int s = j % C::NS;
                 if (j >= C::NS && !mbar_wait(&bars->kv_empty[s], ((j / C::NS) - 1) & 1)) break;
-                mbar_arrive_expect_tx(&bars->k_full[s], C::TILE);
+                mbar_arrive_expect_tx(&bars->k_full[s], C::KTILE);
                 for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_3d(sK + s * C::TILE + hf * C::HALF, &tmK, &bars->k_full[s], hf * 64,
-                                j * C::BN, bh);
-                mbar_arrive_expect_tx(&bars->v_full[s], C::TILE);
+                    tma_load_3d(sK + s * C::KTILE + hf * C::KHALF, &tmK, &bars->k_full[s], hf * 64,
+                                j * BN, bh);
+                mbar_arrive_expect_tx(&bars->v_full[s], C::KTILE);
                 for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_3d(sV + s * C::TILE + hf * C::HALF, &tmV, &bars->v_full[s], hf * 64,
-                                j * C::BN, bh);
+                    tma_load_3d(sV + s * C::VSTAGE + hf * C::KHALF, &tmV, &bars->v_full[s], hf * 64,
+                                j * BN, bh);
             }
         }
     } else if (warp == 5) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0 && T > 0) {
-            constexpr uint32_t kIdescS = idesc_f16(BF16, false, false, 128, 128);
-            constexpr uint32_t kIdescO = idesc_f16(BF16, false, true, 128, D);
-            constexpr uint32_t kIdescSum = idesc_f16(BF16, false, false, 128, 16);
-            const uint64_t ones_desc = smem_desc_sw128(smem_u32(smem + C::OFF_ONES), 16, 1024);
-            const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t k_addr = smem_u32(sK);
-            const uint32_t v_addr = smem_u32(sV);
+            constexpr uint32_t kIdescS = idesc_f16(BF16, false, false, 128, BN);
+            constexpr uint32_t kIdescO = idesc_f16(BF16, false, true, 128, C::PV_N);
+            // Descriptors are built once; per k-step and per stage only the 16-byte start
+            // address field changes, by compile-time offsets.
+            const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t k_desc = smem_desc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t v_desc = smem_desc_sw128(smem_u32(sV), C::KHALF, 1024);
             bool ok = mbar_wait(&bars->q_full, 0);
             tc_fence_after();
             auto issue_s = [&](int j) -> bool {
                 const int s = j % C::NS;
                 if (!mbar_wait(&bars->k_full[s], (j / C::NS) & 1)) return false;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)((j % C::SBUF) * 128);
+                const uint32_t d_tmem = tmem + (uint32_t)((j % C::SBUF) * BN);
+                const uint64_t kd = k_desc + (uint64_t)((s * C::KTILE) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * C::HALF + (kk & 3) * 32);
-                    const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(k_addr + s * C::TILE + off, 16, 1024);
-                    mma_ss(d_tmem, a, bd, kIdescS, kk > 0 ? 1u : 0u);
+                    const uint64_t qo = (uint64_t)(((kk >> 2) * C::QHALF + (kk & 3) * 32) >> 4);
+                    const uint64_t ko = (uint64_t)(((kk >> 2) * C::KHALF + (kk & 3) * 32) >> 4);
+                    mma_ss(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&bars->s_full[j % C::SBUF]);
                 return true;
             };
             if (ok) ok = issue_s(0);
             for (int j = 0; ok && j < T; ++j) {
-                // With two score buffers S_{j+1} goes ahead of P_j V_j; with one it has to
-                // follow it, since P_j lives in the buffer S_{j+1} overwrites.
-                if (C::SBUF == 2 && j + 1 < T && !issue_s(j + 1)) break;
+                if (j + 1 < T) {
+                    if (C::P_OWN) {
+                        // S_{j+1} overwrites S_j as soon as the softmax has read it.
+                        if (!mbar_wait(&bars->s_read, j & 1) || !issue_s(j + 1)) break;
+                    } else if (C::SBUF == 2) {
+                        if (!issue_s(j + 1)) break;  // the other score buffer is free
+                    }
+                }
                 const int s = j % C::NS;
                 if (!mbar_wait(&bars->p_full[j % C::SBUF], (j / C::SBUF) & 1)) break;
                 if (!mbar_wait(&bars->v_full[s], (j / C::NS) & 1)) break;
                 tc_fence_after();
-                const uint32_t p_tmem = tmem + (uint32_t)((j % C::SBUF) * 128);
+                const uint32_t p_tmem =
+                    tmem + (C::P_OWN ? C::COL_P : (uint32_t)((j % C::SBUF) * BN));
+                const uint64_t vd = v_desc + (uint64_t)((s * C::VSTAGE) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t bd =
-                        smem_desc_sw128(v_addr + s * C::TILE + kk * 2048, C::HALF, 1024);
-                    mma_ts(tmem + C::COL_O, p_tmem + kk * 8, bd, kIdescO,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ts(tmem + C::COL_SUM, p_tmem + kk * 8, ones_desc, kIdescSum,
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_ts(tmem + C::COL_O, p_tmem + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), kIdescO,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bars->kv_empty[s]);
                 mma_commit(&bars->o_full);
-                if (C::SBUF == 1 && j + 1 < T && !issue_s(j + 1)) break;
             }
         }
     } else {
@@ -231,34 +257,37 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int j = 0; j < T; ++j) {
             if (!mbar_wait(&bars->s_full[j % C::SBUF], (j / C::SBUF) & 1)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sb = tmem + lane_base + (uint32_t)((j % C::SBUF) * 128);
-            float s[128];
+            const uint32_t sb = tmem + lane_base + (uint32_t)((j % C::SBUF) * BN);
+            float s[BN];
             {
-                uint32_t r[32];
+                uint32_t r[BN];
+                if constexpr (BN == 64) tmem_ld64(sb, r);
+                else tmem_ld128(sb, r);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(sb + c * 32, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-                }
+                for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(r[i]);
             }
-            const bool need_mask = ((j + 1) * C::BN > L) || (p.causal && j == qt);
+            if (C::P_OWN) {
+                tc_fence_before();
+                mbar_arrive(&bars->s_read);
+            }
+            const bool need_mask = ((j + 1) * BN > L) || (p.causal && (j + 1) * BN - 1 > qt * C::BM);
             if (need_mask) {
                 const int lim = p.causal ? min(L, row + 1) : L;  // keys < lim are visible
-                const int c0 = lim - j * C::BN;
+                const int c0 = lim - j * BN;
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
+                for (int c = 0; c < BN; ++c)
                     if (c >= c0) s[c] = -INFINITY;
             }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+            float mxv[8];
 #pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mx0 = fmaxf(mx0, s[c]);
-                mx1 = fmaxf(mx1, s[c + 1]);
-                mx2 = fmaxf(mx2, s[c + 2]);
-                mx3 = fmaxf(mx3, s[c + 3]);
+            for (int c = 0; c < 8; ++c) mxv[c] = s[c];
+#pragma unroll
+            for (int c = 8; c < BN; c += 8) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mxv[e] = fmaxf(mxv[e], s[c + e]);
             }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                                   fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7]))) * sl2;
             // Lazy rescale: move m only when the max grew by more than 2^8.
             const bool grow = mx > m + 8.0f;
             const bool any_grow = __any_sync(0xffffffffu, grow);
@@ -269,9 +298,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             const float m_use = (m == -INFINITY) ? 0.f : m;
             float sum0 = 0.f, sum1 = 0.f;
-            uint32_t pk[64];
+            uint32_t pk[BN / 2];
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
+            for (int c = 0; c < BN; c += 2) {
                 const float p0 = ex2(fmaf(s[c], sl2, -m_use));
                 const float p1 = ex2(fmaf(s[c + 1], sl2, -m_use));
                 sum0 += p0;
@@ -279,24 +308,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 pk[c >> 1] = pack2<BF16>(p0, p1);
             }
             l = l * alpha + (sum0 + sum1);
-            {
-                uint32_t r[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) r[i] = pk[i];
-                tmem_st32(sb, r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) r[i] = pk[32 + i];
-                tmem_st32(sb + 32, r);
-            }
             // Every phase of o_full is waited on, in order, so that a parity wait can
             // never alias a phase two ahead.  P_{j-1} V_{j-1} was issued a whole softmax
-            // block ago, so this wait is normally already satisfied.
+            // block ago, so this wait is normally already satisfied.  It also frees P's
+            // columns (d = 64) before P_j is written there.
             if (j > 0) {
                 if (!mbar_wait(&bars->o_full, (j - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
             }
             if (j > 0 && any_grow) {
-                // Rescale the accumulated output (P_{j-1} V_{j-1} is complete).
+                // Rescale the accumulated output and row sums (P_{j-1} V_{j-1} is done).
                 const uint32_t ob = tmem + lane_base + C::COL_O;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
@@ -312,6 +333,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                     for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
                     tmem_st16(ob + D, r);
+                }
+            }
+            {
+                const uint32_t pb = C::P_OWN ? tmem + lane_base + C::COL_P : sb;
+#pragma unroll
+                for (int h = 0; h < BN / 64; ++h) {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = pk[h * 32 + i];
+                    tmem_st32(pb + h * 32, r);
                 }
             }
             tc_fence_before();
@@ -355,7 +386,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                             __uint_as_float(r[2 * i + 1]) * inv);
             }
             // Row t of this 128-byte column block, 16-byte chunks XOR-swizzled by t % 8.
-            uint8_t *rowp = sQ + hf * C::HALF + t * 128;
+            uint8_t *rowp = sQ + hf * C::QHALF + t * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint4 v4 = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
@@ -366,7 +397,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         named_bar_sync(1, 128);
         if (t == 0) {
             for (int hf = 0; hf < C::HALVES; ++hf)
-                tma_store_3d(&tmO, sQ + hf * C::HALF, hf * 64, qt * C::BM, bh);
+                tma_store_3d(&tmO, sQ + hf * C::QHALF, hf * 64, qt * C::BM, bh);
             bulk_commit_group();
             bulk_wait_group_read<0>();
         }
