@@ -456,33 +456,43 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             // (exactly what the dV MMA consumes; dS below uses the same rounded values).
             uint32_t Pw[32];
             {
-                uint32_t w0[32], w1[32];
-                tmem_ld32(tmem + lane_base + C::COL_S + h * 64, w0);
-                tmem_ld32(tmem + lane_base + C::COL_S + h * 64 + 32, w1);
+                uint32_t w[64];
+                tmem_ld64(tmem + lane_base + C::COL_S + h * 64, w);
                 if (C::P_OWN) {
                     tc_fence_before();
                     mbar_arrive(&bars->s_free);  // S^T may now be overwritten by S_{i+1}
                 }
                 const float *lse2 = sLSE + s * 128 + h * 64;
+                // Masks only on the causal diagonal tile and the key-padding tail tile.
                 const bool diag = p.causal && (qi == kt);
+                const bool tile_masked = diag || (kt * 128 + 128 > L);
+                if (!tile_masked) {
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
+                    for (int k = 0; k < 64; k += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + k);
+                        const float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
+                        const float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
+                        const float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
+                        const float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
+                        Pw[k >> 1] = pack2<BF16>(p0, p1);
+                        Pw[(k >> 1) + 1] = pack2<BF16>(p2, p3);
+                    }
+                } else {
 #pragma unroll
-                    for (int k = 0; k < 32; k += 4) {
-                        const uint32_t *w = cc == 0 ? w0 : w1;
-                        const int c = h * 64 + cc * 32 + k;  // query column in the tile
-                        const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + cc * 32 + k);
+                    for (int k = 0; k < 64; k += 4) {
+                        const int c = h * 64 + k;  // query column in the tile
+                        const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + k);
                         float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
                         float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
                         float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
                         float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
-                        // masked: keys past the valid length, queries before the key (causal)
+                        // keys past the valid length, and queries before the key (causal)
                         if (!key_ok || (diag && c < t)) p0 = 0.f;
                         if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
                         if (!key_ok || (diag && c + 2 < t)) p2 = 0.f;
                         if (!key_ok || (diag && c + 3 < t)) p3 = 0.f;
-                        Pw[cc * 16 + (k >> 1)] = pack2<BF16>(p0, p1);
-                        Pw[cc * 16 + (k >> 1) + 1] = pack2<BF16>(p2, p3);
+                        Pw[k >> 1] = pack2<BF16>(p0, p1);
+                        Pw[(k >> 1) + 1] = pack2<BF16>(p2, p3);
                     }
                 }
             }
@@ -501,10 +511,11 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             tc_fence_after();
             const float *dv = sDv + s * 128 + h * 64;
+            uint32_t wdp[64];
+            tmem_ld64(tmem + lane_base + C::COL_DP + h * 64, wdp);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
-                uint32_t w[32];
-                tmem_ld32(tmem + lane_base + C::COL_DP + h * 64 + cc * 32, w);
+                const uint32_t *w = wdp + cc * 32;
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {

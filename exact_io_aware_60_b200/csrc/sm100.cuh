@@ -157,6 +157,12 @@ __device__ __forceinline__ void bulk_wait_group() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Orders completed async-proxy (TMA) global-memory writes with this thread's later
+// generic-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later async-proxy
 // (TMA, tensor core) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
