@@ -15,7 +15,7 @@
 //      128-row tiles, +inf where there is no row), and zeroes the fp32 dQ accumulator.
 //   2. fa_bwd_kernel: one CTA per 128-key tile of one (batch, head), looping over the
 //      128-query tiles that can see it (causal: only tiles on or below the diagonal).
-//        warp 4      TMA producer: K, V once; Q_i, dO_i (+ LSE_i, D_i) into a 2-stage ring.
+//        warp 8      TMA producer: K, V once; Q_i, dO_i (+ LSE_i, D_i) into a 2/3-stage ring.
 //        warp 5      MMA issuer (one thread), all on tcgen05 with fp32 TMEM accumulators:
 //                    S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i, dK += dS^T Q_i
 //                    (P^T, dS^T read from TMEM), dQ_i = dS K (dS from shared memory).
@@ -142,14 +142,18 @@ struct BwdCfg {
     static constexpr bool P_OWN = (D == 64);
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + TILE;
-    static constexpr int OFF_Q = OFF_V + TILE;       // 2 stages
-    static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // 2 stages
-    static constexpr int OFF_DS = OFF_DO + 2 * TILE; // 128 x 128 16-bit, operand layout
+    // Q_i / dO_i ring: a stage is released only once dQ_i is done, and S_{i+2} needs its
+    // refill right after, so d = 64 keeps three stages to hide the load latency; d = 128
+    // has room for two.
+    static constexpr int QS = (D == 64) ? 3 : 2;
+    static constexpr int OFF_Q = OFF_V + TILE;        // QS stages
+    static constexpr int OFF_DO = OFF_Q + QS * TILE;  // QS stages
+    static constexpr int OFF_DS = OFF_DO + QS * TILE; // 128 x 128 16-bit, operand layout
     static constexpr int OFF_DQ = OFF_DS + 32768;    // fp32 staging (d = 64 only)
     static constexpr int DQ_BYTES = DQ_TMA ? 128 * D * 4 : 0;
-    static constexpr int OFF_LSE = OFF_DQ + DQ_BYTES;  // 2 x 512 B
-    static constexpr int OFF_DV = OFF_LSE + 1024;      // 2 x 512 B
-    static constexpr int OFF_BAR = OFF_DV + 1024;
+    static constexpr int OFF_LSE = OFF_DQ + DQ_BYTES;  // QS x 512 B
+    static constexpr int OFF_DV = OFF_LSE + QS * 512;  // QS x 512 B
+    static constexpr int OFF_BAR = OFF_DV + QS * 512;
     static constexpr int USED = OFF_BAR + 256;
     // d = 128 uses all 227 KB: no room for alignment slack; the kernel checks instead.
     static constexpr int SLACK = (USED + 1024 <= 232448) ? 1024 : 0;
@@ -173,9 +177,9 @@ struct BwdCfg {
 
 struct BwdBars {
     uint64_t kv_full;
-    uint64_t q_full[2];
-    uint64_t do_full[2];
-    uint64_t stage_empty[2];
+    uint64_t q_full[3];
+    uint64_t do_full[3];
+    uint64_t stage_empty[3];
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
         dkv_full;
     uint32_t tmem_base;
@@ -229,7 +233,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tma_prefetch_desc(&tmdV);
         if (C::DQ_TMA) tma_prefetch_desc(&tmdQacc);
         mbar_init(&bars->kv_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::QS; ++i) {
             mbar_init(&bars->q_full[i], 1);
             mbar_init(&bars->do_full[i], 1);
             mbar_init(&bars->stage_empty[i], 1);
@@ -261,9 +265,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tma_load_3d(sV + hf * C::HALF, &tmV, &bars->kv_full, hf * 64, kt * 128, bh);
             }
             for (int i = 0; i < n; ++i) {
-                const int s = i & 1;
+                const int s = i % C::QS;
                 const int qi = q_begin + i;
-                if (i >= 2 && !mbar_wait(&bars->stage_empty[s], ((i >> 1) - 1) & 1)) break;
+                if (i >= C::QS && !mbar_wait(&bars->stage_empty[s], ((i / C::QS) - 1) & 1)) break;
                 const size_t vec_off = (size_t)bh * p.Npad + (size_t)qi * 128;
                 mbar_arrive_expect_tx(&bars->q_full[s], C::TILE + 512);
                 for (int hf = 0; hf < C::HALVES; ++hf)
@@ -326,12 +330,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mma_commit(&bars->dp_full);
             }
             for (int i = 0; ok && i < n; ++i) {
-                const int s = i & 1;
+                const int s = i % C::QS;
                 if (C::P_OWN && i + 1 < n) {
                     // S_{i+1} overwrites S_i as soon as every P/dS warp has read it.
-                    const int s1 = (i + 1) & 1;
+                    const int s1 = (i + 1) % C::QS;
                     if (!mbar_wait(&bars->s_free, i & 1)) break;
-                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
+                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) / C::QS) & 1)) break;
                     tc_fence_after();
                     mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
                     mma_commit(&bars->s_full);
@@ -343,8 +347,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mma_commit(&bars->p_free);
                 if (!C::P_OWN && i + 1 < n) {
                     // P^T_i lives in the S^T columns: S_{i+1} follows dV_i.
-                    const int s1 = (i + 1) & 1;
-                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) >> 1) & 1)) break;
+                    const int s1 = (i + 1) % C::QS;
+                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) / C::QS) & 1)) break;
                     tc_fence_after();
                     mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
                     mma_commit(&bars->s_full);
@@ -365,12 +369,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mma_commit(&bars->ds_empty);
                 mma_commit(&bars->stage_empty[s]);
                 if (i + 1 < n) {
-                    const int s1 = (i + 1) & 1;
+                    const int s1 = (i + 1) % C::QS;
                     if (D == 128) {
                         // dQ_i lives in the dP^T columns: wait until it has been drained.
                         if (!mbar_wait(&bars->dq_empty, i & 1)) break;
                     }
-                    if (!mbar_wait(&bars->do_full[s1], ((i + 1) >> 1) & 1)) break;
+                    if (!mbar_wait(&bars->do_full[s1], ((i + 1) / C::QS) & 1)) break;
                     tc_fence_after();
                     mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
                     mma_commit(&bars->dp_full);
@@ -445,9 +449,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const float sl2 = p.scale_log2;
         bool ok = true;
         for (int i = 0; i < n; ++i) {
-            const int s = i & 1;
+            const int s = i % C::QS;
             const int qi = q_begin + i;
-            if (!mbar_wait(&bars->s_full, i & 1) || !mbar_wait(&bars->q_full[s], (i >> 1) & 1)) {
+            if (!mbar_wait(&bars->s_full, i & 1) || !mbar_wait(&bars->q_full[s], (i / C::QS) & 1)) {
                 ok = false;
                 break;
             }
@@ -504,7 +508,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(&bars->p_full);
 
-            if (!mbar_wait(&bars->dp_full, i & 1) || !mbar_wait(&bars->do_full[s], (i >> 1) & 1) ||
+            if (!mbar_wait(&bars->dp_full, i & 1) || !mbar_wait(&bars->do_full[s], (i / C::QS) & 1) ||
                 (i > 0 && !mbar_wait(&bars->ds_empty, (i - 1) & 1))) {
                 ok = false;
                 break;

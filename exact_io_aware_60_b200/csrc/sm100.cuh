@@ -271,6 +271,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// Two TMEM loads with one wait: 16 columns at `a16` and 32 columns at `a32`.
+__device__ __forceinline__ void tmem_ld16_32(uint32_t a16, uint32_t (&r16)[16], uint32_t a32,
+                                             uint32_t (&r32)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%48];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47}, [%49];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r16[0]), "=r"(r16[1]), "=r"(r16[2]), "=r"(r16[3]), "=r"(r16[4]), "=r"(r16[5]),
+          "=r"(r16[6]), "=r"(r16[7]), "=r"(r16[8]), "=r"(r16[9]), "=r"(r16[10]), "=r"(r16[11]),
+          "=r"(r16[12]), "=r"(r16[13]), "=r"(r16[14]), "=r"(r16[15]), "=r"(r32[0]), "=r"(r32[1]),
+          "=r"(r32[2]), "=r"(r32[3]), "=r"(r32[4]), "=r"(r32[5]), "=r"(r32[6]), "=r"(r32[7]),
+          "=r"(r32[8]), "=r"(r32[9]), "=r"(r32[10]), "=r"(r32[11]), "=r"(r32[12]), "=r"(r32[13]),
+          "=r"(r32[14]), "=r"(r32[15]), "=r"(r32[16]), "=r"(r32[17]), "=r"(r32[18]),
+          "=r"(r32[19]), "=r"(r32[20]), "=r"(r32[21]), "=r"(r32[22]), "=r"(r32[23]),
+          "=r"(r32[24]), "=r"(r32[25]), "=r"(r32[26]), "=r"(r32[27]), "=r"(r32[28]),
+          "=r"(r32[29]), "=r"(r32[30]), "=r"(r32[31])
+        : "r"(a16), "r"(a32)
+        : "memory");
+}
+
 // TMEM -> registers, 32 lanes x 64 consecutive 32-bit columns, single wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
