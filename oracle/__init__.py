@@ -53,6 +53,11 @@ def _load():
             lib.oracle_attention_rows.argtypes = [
                 dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_double, ctypes.c_int,
                 ctypes.c_long, lp, ctypes.c_long, dp, dp, dp, dp, dp]
+            lib.oracle_attention_rows_masked.restype = ctypes.c_int
+            lib.oracle_attention_rows_masked.argtypes = [
+                dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_double, ctypes.c_int,
+                ctypes.c_long, ctypes.c_void_p, ctypes.c_long, lp, ctypes.c_long, dp, dp, dp,
+                dp, dp]
             lib.oracle_threads.restype = ctypes.c_int
             lib.oracle_threads.argtypes = []
             _lib = lib
@@ -76,10 +81,12 @@ def _ptr(a):
 
 
 def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows=None,
-                   want_dkdv=True):
+                   want_dkdv=True, block_mask=None, block_size=128):
     """Exact attention of one (batch, head) for the query rows ``rows``.
 
     q, k, v, dout: ``[N, d]`` arrays (cast to fp64).  ``kv_len``: valid keys (None = N).
+    ``block_mask``: optional ``[nb, nb]`` array (nb = ceil(N / block_size)); key j is
+    visible to query i only where ``block_mask[i // block_size, j // block_size]`` != 0.
     Returns a dict with ``o [R,d]``, ``lse [R]`` and, when ``dout`` is given, ``dq [R,d]``
     and (if ``want_dkdv``) ``dk``, ``dv [N,d]`` summed over the given rows only.
     """
@@ -101,9 +108,15 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
         if want_dkdv:
             dk = np.zeros((N, d))
             dv = np.zeros((N, d))
-    rc = _load().oracle_attention_rows(
+    mask_arr = None
+    if block_mask is not None:
+        nb = (N + block_size - 1) // block_size
+        mask_arr = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+        assert mask_arr.shape == (nb, nb), (mask_arr.shape, nb)
+    rc = _load().oracle_attention_rows_masked(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), N, d, float(scale), int(bool(causal)), L,
-        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), R,
+        None if mask_arr is None else mask_arr.ctypes.data_as(ctypes.c_void_p),
+        int(block_size), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), R,
         _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_rows failed with status {rc}")
@@ -116,11 +129,13 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
     return out
 
 
-def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=None):
+def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=None,
+              block_mask=None, block_size=128):
     """Exact attention over ``[B, H, N, d]`` arrays, one (b, h) at a time.
 
     ``kv_len``: per-batch valid key counts (length B) or None.  ``heads``: optional list
     of (b, h) pairs to evaluate; the others are left as NaN in the outputs.
+    ``block_mask``: optional ``[nb, nb]`` (shared by all heads) or ``[B, H, nb, nb]``.
     Returns ``o``, ``lse`` and, with ``dout``, ``dq``, ``dk``, ``dv`` as fp64 arrays.
     """
     q = np.asarray(q)
@@ -134,8 +149,13 @@ def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=Non
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     for b, h in pairs:
         L = None if kv_len is None else int(kv_len[b])
+        bm = None
+        if block_mask is not None:
+            bm = np.asarray(block_mask)
+            bm = bm if bm.ndim == 2 else bm[b, h]
         r = attention_rows(q[b, h], k[b, h], v[b, h], None if dout is None else dout[b, h],
-                           scale=scale, causal=causal, kv_len=L)
+                           scale=scale, causal=causal, kv_len=L, block_mask=bm,
+                           block_size=block_size)
         o[b, h] = r["o"]
         lse[b, h] = r["lse"]
         if dout is not None:

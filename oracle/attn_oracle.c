@@ -32,7 +32,13 @@
  *   dS_ij = P_ij (dP_ij - D_i)
  *   dQ_i  = scale * sum_j dS_ij k_j
  *   dK_j  = scale * sum_i dS_ij q_i
- * A row with no allowed key (only when L = 0) has O = 0, LSE = -inf, zero gradients.
+ * A row with no allowed key has O = 0, LSE = -inf, zero gradients.
+ *
+ * Block-sparse attention (promptingindex page, "Benchmark results": the same tiling
+ * applied to a sparse pattern; NOTE-005, "Key components": the block-sparse extension)
+ * restricts the allowed set further: with a block mask M of (ceil(N/bs))^2 bytes,
+ *   allowed(i, j) &= M[i / bs][j / bs] != 0,
+ * and is otherwise the same computation.  With M all ones it is dense attention.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -45,9 +51,18 @@
 #define ORACLE_ERR_ARG 1
 #define ORACLE_ERR_NOMEM 2
 
-static int is_allowed(long i, long j, int causal, long L)
+/* Optional block mask (one per (batch, head) call): NULL means dense. */
+typedef struct {
+    const unsigned char *m;
+    long bs; /* block size */
+    long nb; /* blocks per side */
+} block_mask_t;
+
+static int is_allowed(long i, long j, int causal, long L, const block_mask_t *bm)
 {
-    return j < L && (!causal || j <= i);
+    if (!(j < L && (!causal || j <= i))) return 0;
+    if (bm && bm->m) return bm->m[(i / bm->bs) * bm->nb + (j / bm->bs)] != 0;
+    return 1;
 }
 
 /* Rows of the panel processed together.  The score panel holds at most this many
@@ -80,11 +95,21 @@ int oracle_threads(void)
  * dk, dv        : N x d, ACCUMULATED (+=) with the contributions of the given rows, or
  *                 NULL.  Over rows = 0..N-1 they are the full gradients.
  */
-int oracle_attention_rows(const double *q, const double *k, const double *v,
-                          const double *dout, long N, long d, double scale, int causal,
-                          long L, const long *rows, long R, double *o, double *lse,
-                          double *dq, double *dk, double *dv)
+int oracle_attention_rows_masked(const double *q, const double *k, const double *v,
+                                 const double *dout, long N, long d, double scale, int causal,
+                                 long L, const unsigned char *block_mask, long block_size,
+                                 const long *rows, long R, double *o, double *lse, double *dq,
+                                 double *dk, double *dv)
 {
+    block_mask_t bmv;
+    const block_mask_t *bm = NULL;
+    if (block_mask) {
+        if (block_size < 1) return ORACLE_ERR_ARG;
+        bmv.m = block_mask;
+        bmv.bs = block_size;
+        bmv.nb = (N + block_size - 1) / block_size;
+        bm = &bmv;
+    }
     if (!q || !k || !v || !rows || !o || !lse || N < 1 || d < 1 || R < 0 || L < 0 || L > N)
         return ORACLE_ERR_ARG;
     if ((dq || dk || dv) && !dout) return ORACLE_ERR_ARG;
@@ -112,7 +137,7 @@ int oracle_attention_rows(const double *q, const double *k, const double *v,
             /* 1. scaled scores with the mask applied */
             double m = -INFINITY;
             for (long j = 0; j < N; ++j) {
-                if (!is_allowed(i, j, causal, L)) {
+                if (!is_allowed(i, j, causal, L, bm)) {
                     Srow[j] = -INFINITY;
                     continue;
                 }
@@ -156,7 +181,7 @@ int oracle_attention_rows(const double *q, const double *k, const double *v,
             double *dSrow = dS + r * N;
             double D = 0.0;
             for (long j = 0; j < N; ++j) {
-                if (!is_allowed(i, j, causal, L)) {
+                if (!is_allowed(i, j, causal, L, bm)) {
                     dSrow[j] = 0.0;
                     continue;
                 }
@@ -207,4 +232,14 @@ int oracle_attention_rows(const double *q, const double *k, const double *v,
     free(P);
     free(dS);
     return ORACLE_OK;
+}
+
+/* Dense entry point: oracle_attention_rows_masked without a block mask. */
+int oracle_attention_rows(const double *q, const double *k, const double *v,
+                          const double *dout, long N, long d, double scale, int causal,
+                          long L, const long *rows, long R, double *o, double *lse,
+                          double *dq, double *dk, double *dv)
+{
+    return oracle_attention_rows_masked(q, k, v, dout, N, d, scale, causal, L, NULL, 0, rows,
+                                        R, o, lse, dq, dk, dv);
 }

@@ -282,3 +282,96 @@ def test_rejects_bad_arguments():
         oracle.attention_rows(q, q, q, scale=1.0, kv_len=5)
     with pytest.raises(RuntimeError):
         oracle.attention_rows(q, q, q, scale=1.0, rows=np.array([4]))
+
+
+# ---------------------------------------------------------------- block-sparse extension
+
+def brute_force_masked(q, k, v, scale, causal, L, bmask, bs):
+    N = q.shape[0]
+    S = scale * (q @ k.T)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    allowed = (j < L) & ((~np.asarray(causal)) | (j <= i)) & (bmask[i // bs, j // bs] != 0)
+    E = np.where(allowed, np.exp(np.where(allowed, S, 0.0)), 0.0)
+    Z = E.sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        P = np.where(Z[:, None] > 0, E / Z[:, None], 0.0)
+        lse = np.where(Z > 0, np.log(Z), -np.inf)
+    return P @ v, lse
+
+
+@pytest.mark.parametrize("N,bs,causal,L", [(6, 2, False, 6), (7, 2, True, 7), (8, 3, False, 6),
+                                           (8, 2, True, 5), (5, 1, False, 5)])
+def test_block_mask_brute_force(N, bs, causal, L):
+    r = rng(300 + N * bs)
+    d = 3
+    q, k, v = (r.standard_normal((N, d)) for _ in range(3))
+    nb = (N + bs - 1) // bs
+    bmask = (r.random((nb, nb)) < 0.6).astype(np.uint8)
+    res = oracle.attention_rows(q, k, v, scale=0.7, causal=causal, kv_len=L, block_mask=bmask,
+                                block_size=bs)
+    o_bf, lse_bf = brute_force_masked(q, k, v, 0.7, causal, L, bmask, bs)
+    np.testing.assert_allclose(res["o"], o_bf, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(res["lse"], lse_bf, rtol=1e-12, atol=1e-13)
+
+
+def test_block_mask_all_ones_is_dense():
+    N, d = 9, 4
+    r = rng(17)
+    q, k, v, do = (r.standard_normal((N, d)) for _ in range(4))
+    dense = oracle.attention_rows(q, k, v, do, scale=0.5, causal=True, kv_len=8)
+    ones = oracle.attention_rows(q, k, v, do, scale=0.5, causal=True, kv_len=8,
+                                 block_mask=np.ones((3, 3)), block_size=3)
+    for n in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_array_equal(dense[n], ones[n])
+
+
+def test_block_diagonal_mask_factorises():
+    """With only the diagonal blocks allowed, each block of rows is plain attention over
+    its own block of keys."""
+    N, d, bs = 8, 3, 4
+    r = rng(18)
+    q, k, v, do = (r.standard_normal((N, d)) for _ in range(4))
+    res = oracle.attention_rows(q, k, v, do, scale=0.9, block_mask=np.eye(2), block_size=bs)
+    for b in range(2):
+        sl = slice(b * bs, (b + 1) * bs)
+        part = oracle.attention_rows(q[sl], k[sl], v[sl], do[sl], scale=0.9)
+        for n in ("o", "lse", "dq"):
+            np.testing.assert_allclose(res[n][sl], part[n], atol=1e-14)
+        for n in ("dk", "dv"):
+            np.testing.assert_allclose(res[n][sl], part[n], atol=1e-14)
+
+
+def test_block_mask_empty_rows():
+    N, d = 6, 2
+    r = rng(19)
+    q, k, v, do = (r.standard_normal((N, d)) for _ in range(4))
+    bmask = np.array([[0, 0, 0], [1, 1, 0], [0, 1, 1]])
+    res = oracle.attention_rows(q, k, v, do, scale=1.0, block_mask=bmask, block_size=2)
+    assert np.all(res["o"][:2] == 0) and np.all(np.isneginf(res["lse"][:2]))
+    assert np.all(res["dq"][:2] == 0)
+    assert np.all(np.isfinite(res["lse"][2:]))
+
+
+def test_block_mask_gradients_vs_central_differences():
+    N, d, bs = 6, 2, 2
+    r = rng(20)
+    q, k, v, do = (r.standard_normal((N, d)) for _ in range(4))
+    bmask = np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]])
+    kw = dict(scale=0.8, causal=False, block_mask=bmask, block_size=bs)
+    res = oracle.attention_rows(q, k, v, do, **kw)
+
+    def L(qq, kk, vv):
+        return float(np.sum(oracle.attention_rows(qq, kk, vv, **kw)["o"] * do))
+
+    eps = 1e-6
+    for name, idx in (("dq", 0), ("dk", 1), ("dv", 2)):
+        args = [q, k, v]
+        fd = np.zeros((N, d))
+        for pos in np.ndindex(N, d):
+            ap = [a.copy() for a in args]
+            am = [a.copy() for a in args]
+            ap[idx][pos] += eps
+            am[idx][pos] -= eps
+            fd[pos] = (L(*ap) - L(*am)) / (2 * eps)
+        assert np.linalg.norm(res[name] - fd) <= 1e-7 * max(np.linalg.norm(fd), 1.0), name
