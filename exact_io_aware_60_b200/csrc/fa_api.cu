@@ -127,7 +127,8 @@ cudaError_t set_smem(K kern, int bytes, std::atomic<int> *done, int dev) {
 
 template <int D, bool BF16>
 int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
-               int N, float scale, int causal, const int *kv_len, cudaStream_t st, int dev) {
+               int N, float scale, int causal, const int *kv_len, const uint8_t *bmask,
+               int mask_per_head, cudaStream_t st, int dev) {
     using C = fa::FwdCfg<D>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -141,6 +142,9 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     fa::FwdParams p;
     p.lse = lse;
     p.kv_len = kv_len;
+    p.bmask = bmask;
+    p.bmask_T = (N + 127) / 128;
+    p.bmask_bh_stride = mask_per_head ? (long long)p.bmask_T * p.bmask_T : 0;
     p.N = N;
     p.BH = (int)bh;
     p.H = H;
@@ -200,7 +204,8 @@ int grid_for(long long work, int threads) {
 template <int D, bool BF16>
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
                const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, float scale,
-               int causal, const int *kv_len, void *workspace, cudaStream_t st, int dev) {
+               int causal, const int *kv_len, const uint8_t *bmask, int mask_per_head,
+               void *workspace, cudaStream_t st, int dev) {
     using C = fa::BwdCfg<D>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -244,6 +249,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.lse2 = ws.lse2;
     p.dvec = ws.dvec;
     p.dq_acc = ws.dq_acc;
+    p.bmask = bmask;
+    p.bmask_bh_stride = mask_per_head ? (long long)num_tiles * num_tiles : 0;
     p.kv_len = kv_len;
     p.N = N;
     p.Npad = num_tiles * 128;
@@ -333,8 +340,9 @@ const char *fa_strerror(int status) {
 
 const char *fa_last_cuda_error(void) { return t_last_error; }
 
-int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
-           int d, float scale, int causal, const int *kv_len, int dtype, void *stream) {
+static int fwd_common(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                      int H, int N, int d, float scale, int causal, const int *kv_len,
+                      const uint8_t *bmask, int mask_per_head, int dtype, void *stream) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_INVALID_ARG;
@@ -346,11 +354,26 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
+#define FA_FWD_ARGS q, k, v, o, lse, B, H, N, scale, causal, kv_len, bmask, mask_per_head, st, dev
     if (d == 64)
-        return bf16 ? launch_fwd<64, true>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev)
-                    : launch_fwd<64, false>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev);
-    return bf16 ? launch_fwd<128, true>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev)
-                : launch_fwd<128, false>(q, k, v, o, lse, B, H, N, scale, causal, kv_len, st, dev);
+        return bf16 ? launch_fwd<64, true>(FA_FWD_ARGS) : launch_fwd<64, false>(FA_FWD_ARGS);
+    return bf16 ? launch_fwd<128, true>(FA_FWD_ARGS) : launch_fwd<128, false>(FA_FWD_ARGS);
+#undef FA_FWD_ARGS
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
+           int d, float scale, int causal, const int *kv_len, int dtype, void *stream) {
+    return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, nullptr, 0, dtype,
+                      stream);
+}
+
+int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                       int H, int N, int d, float scale, int causal, const int *kv_len,
+                       const unsigned char *block_mask, int mask_per_head, int dtype,
+                       void *stream) {
+    if (!block_mask || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
+    return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, block_mask,
+                      mask_per_head, dtype, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -358,10 +381,11 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
     return bwd_workspace_layout(nullptr, (long long)B * H, N, d).total;
 }
 
-int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
-           const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
-           float scale, int causal, const int *kv_len, int dtype, void *workspace,
-           size_t workspace_bytes, void *stream) {
+static int bwd_common(const void *q, const void *k, const void *v, const void *o,
+                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                      int H, int N, int d, float scale, int causal, const int *kv_len,
+                      const uint8_t *bmask, int mask_per_head, int dtype, void *workspace,
+                      size_t workspace_bytes, void *stream) {
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
         return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
@@ -377,11 +401,29 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
-#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, workspace, st, dev
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, bmask, mask_per_head, workspace, st, dev
     if (d == 64)
         return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
     return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
 #undef FA_BWD_ARGS
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+           float scale, int causal, const int *kv_len, int dtype, void *workspace,
+           size_t workspace_bytes, void *stream) {
+    return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, kv_len,
+                      nullptr, 0, dtype, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
+                       const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                       int H, int N, int d, float scale, int causal, const int *kv_len,
+                       const unsigned char *block_mask, int mask_per_head, int dtype,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (!block_mask || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
+    return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, kv_len,
+                      block_mask, mask_per_head, dtype, workspace, workspace_bytes, stream);
 }
 
 int fa_selftest_wait_timeout(int limit_us, void *stream) {
@@ -418,7 +460,7 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, c
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
-#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, workspace, st, dev
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, nullptr, 0, workspace, st, dev
     if (d == 64)
         return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
     return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);

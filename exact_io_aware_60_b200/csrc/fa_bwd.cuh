@@ -118,6 +118,10 @@ __global__ void __launch_bounds__(256) fa_bwd_convert_kernel(const float4 *acc, 
 
 struct BwdParams {
     const float *lse2;  // [BH][Npad], log2-domain LSE (+inf for padding rows)
+    // Block-sparse attention: uint8 [heads][T][T]; key tile kt visits only the query tiles
+    // qi with mask[qi][kt] != 0.  nullptr = dense.
+    const uint8_t *bmask;
+    long long bmask_bh_stride;  // 0: one mask for every (batch, head)
     const float *dvec;  // [BH][Npad]
     float *dq_acc;      // [BH][N][D] fp32
     const int *kv_len;
@@ -222,7 +226,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         L = L < 0 ? 0 : (L > p.N ? p.N : L);
     }
     const int q_begin = p.causal ? kt : 0;
-    const int n = (kt * 128 < L) ? (p.num_tiles - q_begin) : 0;  // query tiles visited
+    // Block-sparse walk: next query tile at or after qi whose (qi, kt) entry is set.
+    const uint8_t *mcol = p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + kt : nullptr;
+    auto next_q = [&](int qi) -> int {
+        if (mcol)
+            while (qi < p.num_tiles && mcol[(size_t)qi * p.num_tiles] == 0) ++qi;
+        return qi;
+    };
+    const int q_first = next_q(q_begin);
+    int n = 0;  // query tiles visited
+    if (kt * 128 < L)
+        for (int qi = q_first; qi < p.num_tiles; qi = next_q(qi + 1)) ++n;
 
     if (warp == C::W_TMA && lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -264,9 +278,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tma_load_3d(sK + hf * C::HALF, &tmK, &bars->kv_full, hf * 64, kt * 128, bh);
                 tma_load_3d(sV + hf * C::HALF, &tmV, &bars->kv_full, hf * 64, kt * 128, bh);
             }
-            for (int i = 0; i < n; ++i) {
+            for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
                 const int s = i % C::QS;
-                const int qi = q_begin + i;
                 if (i >= C::QS && !mbar_wait(&bars->stage_empty[s], ((i / C::QS) - 1) & 1)) break;
                 const size_t vec_off = (size_t)bh * p.Npad + (size_t)qi * 128;
                 mbar_arrive_expect_tx(&bars->q_full[s], C::TILE + 512);
@@ -388,8 +401,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int r = quarter * 32 + lane;          // query row in the tile = TMEM lane
         const int gt = threadIdx.x - C::W_DQ0 * 32;  // 0..127 inside this warpgroup
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        for (int i = 0; i < n; ++i) {
-            const int qi = q_begin + i;
+        for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
             if (!mbar_wait(&bars->dq_full, i & 1)) break;
             tc_fence_after();
             if constexpr (C::DQ_TMA) {
@@ -448,9 +460,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
-        for (int i = 0; i < n; ++i) {
+        for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
             const int s = i % C::QS;
-            const int qi = q_begin + i;
             if (!mbar_wait(&bars->s_full, i & 1) || !mbar_wait(&bars->q_full[s], (i / C::QS) & 1)) {
                 ok = false;
                 break;

@@ -35,6 +35,10 @@
 // A tcgen05.mma instruction costs at least ~45 cycles whatever its N, so small MMAs are
 // merged where possible (the row sums ride on the PV instruction).
 //
+// Block-sparse attention (promptingindex page, "Benchmark results"; NOTE-005, "Key
+// components"): with a block mask, every role walks only the key blocks whose 128 x 128
+// (query tile, key tile) entry is set; skipped blocks cost nothing.
+//
 // The loop order is query-block outer (each CTA writes its O rows once) instead of the
 // key-block-outer order of the original algorithm; the result is the same up to
 // floating-point ordering.
@@ -49,6 +53,11 @@ namespace fa {
 struct FwdParams {
     float *lse;
     const int *kv_len;
+    // Block-sparse attention: uint8 [heads][T128][T128] (T128 = ceil(N / 128)); a query
+    // tile visits only key tiles whose byte is nonzero.  nullptr = dense.
+    const uint8_t *bmask;
+    long long bmask_bh_stride;  // 0: one mask for every (batch, head)
+    int bmask_T;
     int N;
     int BH;
     int H;
@@ -138,7 +147,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     int kv_end = L;
     if (p.causal) kv_end = min(kv_end, (qt + 1) * C::BM);
-    const int T = (kv_end + BN - 1) / BN;  // key blocks this tile visits
+    const int T = (kv_end + BN - 1) / BN;  // key blocks in range
+    // Block-sparse walk: next key block at or after j whose tile is set (T if none).
+    const uint8_t *mrow =
+        p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + (size_t)qt * p.bmask_T : nullptr;
+    auto next_block = [&](int j) -> int {
+        if (mrow)
+            while (j < T && mrow[(j * BN) >> 7] == 0) ++j;
+        return j;
+    };
+    const int j_first = next_block(0);
+    const bool any_block = j_first < T;
 
     if (threadIdx.x == 128) {
         tma_prefetch_desc(&tmQ);
@@ -176,13 +195,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     if (warp == 4) {
         // ------------------------------ TMA producer ------------------------------
-        if (lane == 0 && T > 0) {
+        if (lane == 0 && any_block) {
             mbar_arrive_expect_tx(&bars->q_full, C::QTILE);
             for (int hf = 0; hf < C::HALVES; ++hf)
                 tma_load_3d(sQ + hf * C::QHALF, &tmQ, &bars->q_full, hf * 64, qt * C::BM, bh);
-            for (int j = 0; j < T; ++j) {
-                const int s = j % C::NS;
-                if (j >= C::NS && !mbar_wait(&bars->kv_empty[s], ((j / C::NS) - 1) & 1)) break;
+            int jj = 0;  // index among the visited blocks: drives stages and phases
+            for (int j = j_first; j < T; j = next_block(j + 1), ++jj) {
+                const int s = jj % C::NS;
+                if (jj >= C::NS && !mbar_wait(&bars->kv_empty[s], ((jj / C::NS) - 1) & 1)) break;
                 mbar_arrive_expect_tx(&bars->k_full[s], C::KTILE);
                 for (int hf = 0; hf < C::HALVES; ++hf)
                     tma_load_3d(sK + s * C::KTILE + hf * C::KHALF, &tmK, &bars->k_full[s], hf * 64,
@@ -195,7 +215,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
     } else if (warp == 5) {
         // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0 && T > 0) {
+        if (lane == 0 && any_block) {
             constexpr uint32_t kIdescS = idesc_f16(BF16, false, false, 128, BN);
             constexpr uint32_t kIdescO = idesc_f16(BF16, false, true, 128, C::PV_N);
             // Descriptors are built once; per k-step and per stage only the 16-byte start
@@ -205,11 +225,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint64_t v_desc = smem_desc_sw128(smem_u32(sV), C::KHALF, 1024);
             bool ok = mbar_wait(&bars->q_full, 0);
             tc_fence_after();
-            auto issue_s = [&](int j) -> bool {
-                const int s = j % C::NS;
-                if (!mbar_wait(&bars->k_full[s], (j / C::NS) & 1)) return false;
+            // jj: index of the visited block (stages, phases and buffers follow it)
+            auto issue_s = [&](int jj) -> bool {
+                const int s = jj % C::NS;
+                if (!mbar_wait(&bars->k_full[s], (jj / C::NS) & 1)) return false;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)((j % C::SBUF) * BN);
+                const uint32_t d_tmem = tmem + (uint32_t)((jj % C::SBUF) * BN);
                 const uint64_t kd = k_desc + (uint64_t)((s * C::KTILE) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -217,32 +238,35 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const uint64_t ko = (uint64_t)(((kk >> 2) * C::KHALF + (kk & 3) * 32) >> 4);
                     mma_ss(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full[j % C::SBUF]);
+                mma_commit(&bars->s_full[jj % C::SBUF]);
                 return true;
             };
             if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < T; ++j) {
-                if (j + 1 < T) {
+            int jj = 0;
+            for (int j = j_first; ok && j < T; ++jj) {
+                const int jn = next_block(j + 1);
+                if (jn < T) {
                     if (C::P_OWN) {
-                        // S_{j+1} overwrites S_j as soon as the softmax has read it.
-                        if (!mbar_wait(&bars->s_read, j & 1) || !issue_s(j + 1)) break;
+                        // S_{jj+1} overwrites S_jj as soon as the softmax has read it.
+                        if (!mbar_wait(&bars->s_read, jj & 1) || !issue_s(jj + 1)) break;
                     } else if (C::SBUF == 2) {
-                        if (!issue_s(j + 1)) break;  // the other score buffer is free
+                        if (!issue_s(jj + 1)) break;  // the other score buffer is free
                     }
                 }
-                const int s = j % C::NS;
-                if (!mbar_wait(&bars->p_full[j % C::SBUF], (j / C::SBUF) & 1)) break;
-                if (!mbar_wait(&bars->v_full[s], (j / C::NS) & 1)) break;
+                const int s = jj % C::NS;
+                if (!mbar_wait(&bars->p_full[jj % C::SBUF], (jj / C::SBUF) & 1)) break;
+                if (!mbar_wait(&bars->v_full[s], (jj / C::NS) & 1)) break;
                 tc_fence_after();
                 const uint32_t p_tmem =
-                    tmem + (C::P_OWN ? C::COL_P : (uint32_t)((j % C::SBUF) * BN));
+                    tmem + (C::P_OWN ? C::COL_P : (uint32_t)((jj % C::SBUF) * BN));
                 const uint64_t vd = v_desc + (uint64_t)((s * C::VSTAGE) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
                     mma_ts(tmem + C::COL_O, p_tmem + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), kIdescO,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                           (jj > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bars->kv_empty[s]);
                 mma_commit(&bars->o_full);
+                j = jn;
             }
         }
     } else {
@@ -254,10 +278,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float m = -INFINITY;  // running max, in units of log2 (already scaled)
         float l = 0.f;        // running normaliser
         bool ok = true;
-        for (int j = 0; j < T; ++j) {
-            if (!mbar_wait(&bars->s_full[j % C::SBUF], (j / C::SBUF) & 1)) { ok = false; break; }
+        int jj = 0;  // visited blocks so far
+        for (int j = j_first; j < T; j = next_block(j + 1), ++jj) {
+            if (!mbar_wait(&bars->s_full[jj % C::SBUF], (jj / C::SBUF) & 1)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sb = tmem + lane_base + (uint32_t)((j % C::SBUF) * BN);
+            const uint32_t sb = tmem + lane_base + (uint32_t)((jj % C::SBUF) * BN);
             float s[BN];
             {
                 uint32_t r[BN];
@@ -312,11 +337,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             // never alias a phase two ahead.  P_{j-1} V_{j-1} was issued a whole softmax
             // block ago, so this wait is normally already satisfied.  It also frees P's
             // columns (d = 64) before P_j is written there.
-            if (j > 0) {
-                if (!mbar_wait(&bars->o_full, (j - 1) & 1)) { ok = false; break; }
+            if (jj > 0) {
+                if (!mbar_wait(&bars->o_full, (jj - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
             }
-            if (j > 0 && any_grow) {
+            if (jj > 0 && any_grow) {
                 // Rescale the accumulated output and row sums (P_{j-1} V_{j-1} is done).
                 const uint32_t ob = tmem + lane_base + C::COL_O;
 #pragma unroll
@@ -346,17 +371,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->p_full[j % C::SBUF]);
+            mbar_arrive(&bars->p_full[jj % C::SBUF]);
         }
 
         // ------------------------------ epilogue ------------------------------
-        if (ok && T > 0) {
-            ok = mbar_wait(&bars->o_full, (T - 1) & 1);
+        if (ok && jj > 0) {
+            ok = mbar_wait(&bars->o_full, (jj - 1) & 1);
             tc_fence_after();
         }
         const uint32_t ob = tmem + lane_base + C::COL_O;
         float l_round = 0.f;
-        if (T > 0) {
+        if (any_block) {
             uint32_t r[16];
             tmem_ld16(ob + D, r);
             l_round = __uint_as_float(r[0]);
@@ -367,7 +392,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             uint32_t w[32];
             {
                 uint32_t r[32];
-                if (T > 0) {
+                if (any_block) {
                     tmem_ld32(ob + hf * 64, r);
                 } else {
 #pragma unroll
@@ -377,7 +402,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int i = 0; i < 16; ++i)
                     w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv,
                                        __uint_as_float(r[2 * i + 1]) * inv);
-                if (T > 0) {
+                if (any_block) {
                     tmem_ld32(ob + hf * 64 + 32, r);
                 }
 #pragma unroll

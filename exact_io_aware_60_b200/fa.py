@@ -71,6 +71,12 @@ def lib():
             L.fa_set_timing_events.argtypes = [i, vp, vp]
             L.fa_selftest_wait_timeout.restype = i
             L.fa_selftest_wait_timeout.argtypes = [i, vp]
+            L.fa_fwd_blocksparse.restype = i
+            L.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, i, i,
+                                             vp]
+            L.fa_bwd_blocksparse.restype = i
+            L.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f,
+                                             i, vp, vp, i, i, vp, sz, vp]
             L.fa_bwd_noalloc.restype = i
             L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i,
                                          vp, i, vp]
@@ -158,6 +164,59 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: bool = Fa
                       workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
+
+
+def _mask_args(block_mask, B, H, N):
+    T = (N + 127) // 128
+    if not isinstance(block_mask, torch.Tensor) or not block_mask.is_cuda:
+        raise FAError(FA_ERR_INVALID_ARG, "block_mask must be a CUDA tensor")
+    if block_mask.dtype != torch.uint8 or not block_mask.is_contiguous():
+        raise FAError(FA_ERR_INVALID_ARG, "block_mask must be a contiguous uint8 tensor")
+    if tuple(block_mask.shape) == (T, T):
+        return block_mask.data_ptr(), 0
+    if tuple(block_mask.shape) == (B, H, T, T):
+        return block_mask.data_ptr(), 1
+    raise FAError(FA_ERR_INVALID_ARG,
+                  f"block_mask shape must be ({T}, {T}) or ({B}, {H}, {T}, {T})")
+
+
+def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, *, scale: float, causal: bool = False,
+                       kv_len=None, stream=None) -> None:
+    """Block-sparse forward: ``block_mask`` is a uint8 CUDA tensor [T, T] or [B, H, T, T]
+    (T = ceil(N/128)); key tile kt is visible to query tile qt only where it is nonzero."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    mp, per_head = _mask_args(block_mask, B, H, N)
+    rc = lib().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                                  _kv_ptr(kv_len, B), mp, per_head, _dtype_code(q),
+                                  _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_blocksparse")
+
+
+def fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, block_mask, *, scale: float,
+                       causal: bool = False, kv_len=None, workspace: torch.Tensor,
+                       stream=None) -> None:
+    """Block-sparse backward with the same ``block_mask`` as the forward call."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise FAError(FA_ERR_INVALID_ARG, "workspace must be a contiguous uint8 CUDA tensor")
+    mp, per_head = _mask_args(block_mask, B, H, N)
+    rc = lib().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                  dv.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                                  _kv_ptr(kv_len, B), mp, per_head, _dtype_code(q),
+                                  workspace.data_ptr(), workspace.numel(),
+                                  _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_blocksparse")
 
 
 def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: bool = False,

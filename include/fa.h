@@ -129,6 +129,35 @@ FA_API const char *fa_last_cuda_error(void);
 FA_API int fa_get_device_status(void *stream);
 
 /*
+ * Block-sparse attention (promptingindex page, "Benchmark results": the same tiling
+ * applied to sparse patterns; NOTE-005, "Key components" and "Limitations": the
+ * block-sparse extension, which is exact for its pattern and approximate as a stand-in
+ * for dense attention).  Identical to fa_fwd / fa_bwd except that key j is visible to
+ * query i only if, in addition to the Mask rule above,
+ *     block_mask[i / 128][j / 128] != 0.
+ * Skipped blocks are neither loaded nor multiplied.
+ *   block_mask    : DEVICE pointer to uint8 [T][T] (T = ceil(N / 128)), row = query tile,
+ *                   column = key tile; with mask_per_head = 1, [B * H][T][T] (index
+ *                   b * H + h).  Read only.
+ *   mask_per_head : 0 (one mask for every batch and head) or 1.
+ * Rows whose visible set is empty get O = 0, LSE = -inf and zero gradients.  The backward
+ * call must be given the same mask as the forward call that produced o and lse.
+ * Returns FA_ERR_INVALID_ARG for a null mask or a bad mask_per_head; otherwise as fa_fwd /
+ * fa_bwd.
+ */
+FA_API int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                              int B, int H, int N, int d, float scale, int causal,
+                              const int *kv_len, const unsigned char *block_mask,
+                              int mask_per_head, int dtype, void *stream);
+
+FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
+                              const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                              int B, int H, int N, int d, float scale, int causal,
+                              const int *kv_len, const unsigned char *block_mask,
+                              int mask_per_head, int dtype, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
  * Backward pass for callers that cannot allocate device memory.  The FlashAttention
  * pages have no counterpart to this entry point: it exists for the environment, not the
  * method.  Some hosts of this library may not call cudaMalloc at all: plugins inside

@@ -45,11 +45,13 @@ def run_gpu(inp: dict, scale: float, causal: bool, backward: bool = True):
     return {n: t.cpu() for n, t in out.items()}
 
 
-def oracle_full(inp: dict, scale: float, causal: bool, backward: bool = True, heads=None):
+def oracle_full(inp: dict, scale: float, causal: bool, backward: bool = True, heads=None,
+                block_mask=None):
     q, k, v = (to_f64(inp[n]) for n in ("q", "k", "v"))
     do = to_f64(inp["do"]) if backward else None
     kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
-    return oracle.attention(q, k, v, do, scale=scale, causal=causal, kv_len=kv, heads=heads)
+    return oracle.attention(q, k, v, do, scale=scale, causal=causal, kv_len=kv, heads=heads,
+                            block_mask=block_mask, block_size=128)
 
 
 def lse_err(gpu_lse: np.ndarray, ref_lse: np.ndarray) -> float:

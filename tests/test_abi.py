@@ -110,3 +110,17 @@ def test_binding_raises_without_cuda_tensors():
     x = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(fa.FAError):
         fa.fa_fwd(x, x, x, x, torch.zeros(1, 1, 4), scale=0.1)
+
+
+def test_blocksparse_rejects_missing_or_bad_mask():
+    L = fa.lib()
+    a = dict(GOOD)
+    rc = L.fa_fwd_blocksparse(P, P, P, P, P, a["B"], a["H"], a["N"], a["d"], a["scale"], 0,
+                              None, None, 0, 0, None)
+    assert rc == fa.FA_ERR_INVALID_ARG
+    rc = L.fa_fwd_blocksparse(P, P, P, P, P, a["B"], a["H"], a["N"], a["d"], a["scale"], 0,
+                              None, P, 2, 0, None)
+    assert rc == fa.FA_ERR_INVALID_ARG
+    rc = L.fa_bwd_blocksparse(P, P, P, P, P, P, P, P, P, a["B"], a["H"], a["N"], a["d"],
+                              a["scale"], 0, None, None, 0, 0, P * 16, 1 << 30, None)
+    assert rc == fa.FA_ERR_INVALID_ARG
