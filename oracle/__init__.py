@@ -12,7 +12,10 @@ That Rewrote GPU Training Speed Records", section "Tiling").  This module only m
 numpy arrays into it.
 
 Pins: every function here is pinned by ``tests/test_oracle_pins.py`` (brute-force
-softmax without max shift, closed forms, invariants, central finite differences).
+softmax without max shift, closed forms, invariants, central finite differences) and,
+for dropout and its random numbers, by ``tests/test_oracle_dropout_pins.py`` (published
+Philox4x32-10 known-answer vectors, cuRAND's host Philox generator, statistics of the
+mask, finite differences through a fixed mask).
 """
 from __future__ import annotations
 
@@ -41,6 +44,11 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+class _Dropout(ctypes.Structure):
+    _fields_ = [("threshold", ctypes.c_uint), ("seed", ctypes.c_ulonglong),
+                ("offset", ctypes.c_uint), ("bh", ctypes.c_uint)]
+
+
 def _load():
     global _lib
     with _lock:
@@ -58,6 +66,21 @@ def _load():
                 dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_double, ctypes.c_int,
                 ctypes.c_long, ctypes.c_void_p, ctypes.c_long, lp, ctypes.c_long, dp, dp, dp,
                 dp, dp]
+            lib.oracle_attention_rows_ex.restype = ctypes.c_int
+            lib.oracle_attention_rows_ex.argtypes = [
+                dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_double, ctypes.c_int,
+                ctypes.c_long, ctypes.c_void_p, ctypes.c_long, ctypes.POINTER(_Dropout), lp,
+                ctypes.c_long, dp, dp, dp, dp, dp]
+            u32p = ctypes.POINTER(ctypes.c_uint)
+            lib.oracle_philox4x32_10.restype = None
+            lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+            lib.oracle_dropout_byte.restype = ctypes.c_uint
+            lib.oracle_dropout_byte.argtypes = [ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_uint,
+                                                ctypes.c_long, ctypes.c_long]
+            lib.oracle_dropout_keep.restype = ctypes.c_int
+            lib.oracle_dropout_keep.argtypes = [ctypes.c_uint, ctypes.c_ulonglong, ctypes.c_uint,
+                                                ctypes.c_uint, ctypes.c_long, ctypes.c_long,
+                                                ctypes.c_void_p]
             lib.oracle_threads.restype = ctypes.c_int
             lib.oracle_threads.argtypes = []
             _lib = lib
@@ -67,6 +90,42 @@ def _load():
 def threads() -> int:
     """OpenMP threads the oracle uses."""
     return int(_load().oracle_threads())
+
+
+def dropout_threshold(p) -> int:
+    """Byte threshold t of drop probability ``p``: p is taken in single precision and
+    rounded to the nearest multiple of 1/256 (ties to even); a random byte below t drops
+    the element, so the drop probability used is exactly t / 256.  Valid for 0 <= t < 256.
+    """
+    t = int(np.rint(np.float32(p) * np.float32(256.0)))
+    if not (0 <= t < 256):
+        raise ValueError(f"dropout probability {p} is outside [0, 255.5/256)")
+    return t
+
+
+def philox4x32_10(ctr, key):
+    """The four 32-bit output words of Philox4x32-10 for counter ``ctr`` (4 words) and
+    key ``key`` (2 words)."""
+    c = (ctypes.c_uint * 4)(*[int(x) & 0xFFFFFFFF for x in ctr])
+    k = (ctypes.c_uint * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+    o = (ctypes.c_uint * 4)()
+    _load().oracle_philox4x32_10(c, k, o)
+    return [int(x) for x in o]
+
+
+def dropout_byte(seed, offset, bh, i, j) -> int:
+    """The random byte that decides element (i, j) of head ``bh``."""
+    return int(_load().oracle_dropout_byte(int(seed), int(offset), int(bh), int(i), int(j)))
+
+
+def dropout_keep(p, seed, offset, bh, n_q, n_k):
+    """Keep mask ``[n_q, n_k]`` (uint8, 1 = kept) of head ``bh`` (= b * H + h)."""
+    keep = np.zeros((n_q, n_k), dtype=np.uint8)
+    rc = _load().oracle_dropout_keep(dropout_threshold(p), int(seed), int(offset), int(bh),
+                                     n_q, n_k, keep.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise RuntimeError(f"oracle_dropout_keep failed with status {rc}")
+    return keep
 
 
 def _f64(a):
@@ -81,12 +140,15 @@ def _ptr(a):
 
 
 def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows=None,
-                   want_dkdv=True, block_mask=None, block_size=128):
+                   want_dkdv=True, block_mask=None, block_size=128, dropout_p=0.0, seed=0,
+                   offset=0, bh=0):
     """Exact attention of one (batch, head) for the query rows ``rows``.
 
     q, k, v, dout: ``[N, d]`` arrays (cast to fp64).  ``kv_len``: valid keys (None = N).
     ``block_mask``: optional ``[nb, nb]`` array (nb = ceil(N / block_size)); key j is
     visible to query i only where ``block_mask[i // block_size, j // block_size]`` != 0.
+    ``dropout_p``, ``seed``, ``offset``, ``bh``: dropout on the probabilities with the
+    counter-based mask of head ``bh`` (see ``dropout_keep``); 0 = no dropout.
     Returns a dict with ``o [R,d]``, ``lse [R]`` and, when ``dout`` is given, ``dq [R,d]``
     and (if ``want_dkdv``) ``dk``, ``dv [N,d]`` summed over the given rows only.
     """
@@ -113,11 +175,12 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
         nb = (N + block_size - 1) // block_size
         mask_arr = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
         assert mask_arr.shape == (nb, nb), (mask_arr.shape, nb)
-    rc = _load().oracle_attention_rows_masked(
+    drop = _Dropout(dropout_threshold(dropout_p), int(seed), int(offset), int(bh))
+    rc = _load().oracle_attention_rows_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), N, d, float(scale), int(bool(causal)), L,
         None if mask_arr is None else mask_arr.ctypes.data_as(ctypes.c_void_p),
-        int(block_size), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), R,
-        _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv))
+        int(block_size), ctypes.byref(drop), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)),
+        R, _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_rows failed with status {rc}")
     out = {"o": o, "lse": lse}
@@ -130,12 +193,13 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
 
 
 def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=None,
-              block_mask=None, block_size=128):
+              block_mask=None, block_size=128, dropout_p=0.0, seed=0, offset=0):
     """Exact attention over ``[B, H, N, d]`` arrays, one (b, h) at a time.
 
     ``kv_len``: per-batch valid key counts (length B) or None.  ``heads``: optional list
     of (b, h) pairs to evaluate; the others are left as NaN in the outputs.
     ``block_mask``: optional ``[nb, nb]`` (shared by all heads) or ``[B, H, nb, nb]``.
+    ``dropout_p``, ``seed``, ``offset``: dropout, head (b, h) drawing its mask as bh = b*H+h.
     Returns ``o``, ``lse`` and, with ``dout``, ``dq``, ``dk``, ``dv`` as fp64 arrays.
     """
     q = np.asarray(q)
@@ -155,7 +219,8 @@ def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=Non
             bm = bm if bm.ndim == 2 else bm[b, h]
         r = attention_rows(q[b, h], k[b, h], v[b, h], None if dout is None else dout[b, h],
                            scale=scale, causal=causal, kv_len=L, block_mask=bm,
-                           block_size=block_size)
+                           block_size=block_size, dropout_p=dropout_p, seed=seed, offset=offset,
+                           bh=b * H + h)
         o[b, h] = r["o"]
         lse[b, h] = r["lse"]
         if dout is not None:
