@@ -63,9 +63,44 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def step_flops(w) -> tuple:
-    f, b = w.nominal_flops()
-    return f, b, f + b
+def step_flops(w, block_mask=None) -> tuple:
+    """(forward, backward, total) FLOPs of one step.  Dense: the nominal count.  With a
+    block mask: 4 d per visible (query, key) pair forward and 10 d backward (the work the
+    kernels actually do; masked blocks are skipped)."""
+    if block_mask is None:
+        f, b = w.nominal_flops()
+        return f, b, f + b
+    vis = visible_pairs(w.N, block_mask, w.causal)
+    f = 4.0 * w.d * vis * w.B * w.H
+    return f, 2.5 * f, 3.5 * f
+
+
+def local_global_mask(T: int):
+    """Block pattern of the block-sparse measurement: every query tile sees its own and the
+    previous key tile (local band) and the first key tile (global)."""
+    import numpy as np
+    m = np.zeros((T, T), dtype=np.uint8)
+    for i in range(T):
+        m[i, max(0, i - 1):i + 1] = 1
+        m[i, 0] = 1
+    return m
+
+
+def visible_pairs(N: int, mask, causal: bool) -> int:
+    """Number of (query, key) pairs the mask (128 x 128 blocks) and the causal rule allow."""
+    T = mask.shape[0]
+    total = 0
+    for qt in range(T):
+        rows = min(128, N - qt * 128)
+        for kt in range(T):
+            if not mask[qt, kt]:
+                continue
+            cols = min(128, N - kt * 128)
+            if not causal or kt < qt:
+                total += rows * cols
+            elif kt == qt:
+                total += sum(min(r + 1, cols) for r in range(rows))
+    return total
 
 
 def whole_job_tflops(flops_per_step: float, n_gpus: int, steps: int, max_ms: float) -> float:
@@ -206,6 +241,21 @@ def set_bytes(s) -> int:
 
 def run_step(w, s, stream=None):
     from exact_io_aware_60_b200 import fa
+    if s.get("drop") is not None:
+        p, seed = s["drop"]
+        fa.fa_fwd_dropout(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale, p_drop=p,
+                          seed=seed, causal=w.causal, kv_len=s["kv_len"], stream=stream)
+        fa.fa_bwd_dropout(s["q"], s["k"], s["v"], s["o"], s["do"], s["lse"], s["dq"], s["dk"],
+                          s["dv"], scale=w.scale, p_drop=p, seed=seed, causal=w.causal,
+                          kv_len=s["kv_len"], workspace=s["ws"], stream=stream)
+        return
+    if s.get("mask") is not None:
+        fa.fa_fwd_blocksparse(s["q"], s["k"], s["v"], s["o"], s["lse"], s["mask"], scale=w.scale,
+                              causal=w.causal, kv_len=s["kv_len"], stream=stream)
+        fa.fa_bwd_blocksparse(s["q"], s["k"], s["v"], s["o"], s["do"], s["lse"], s["dq"],
+                              s["dk"], s["dv"], s["mask"], scale=w.scale, causal=w.causal,
+                              kv_len=s["kv_len"], workspace=s["ws"], stream=stream)
+        return
     fa.fa_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale, causal=w.causal,
               kv_len=s["kv_len"], stream=stream)
     fa.fa_bwd(s["q"], s["k"], s["v"], s["o"], s["do"], s["lse"], s["dq"], s["dk"], s["dv"],
@@ -213,7 +263,7 @@ def run_step(w, s, stream=None):
               stream=stream)
 
 
-def cpu_baseline_sample(w, inp, budget_s: float) -> dict:
+def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0) -> dict:
     """The oracle (as it stands) on whole heads of the workload until ``budget_s`` of CPU
     time has passed (at least one head)."""
     import oracle
@@ -225,7 +275,8 @@ def cpu_baseline_sample(w, inp, budget_s: float) -> dict:
     for b, h in heads:
         L = w.N if kv is None else int(kv[b])
         oracle.attention_rows(q[b, h], k[b, h], v[b, h], do[b, h], scale=w.scale,
-                              causal=w.causal, kv_len=L)
+                              causal=w.causal, kv_len=L, dropout_p=dropout_p, seed=1234,
+                              bh=b * w.H + h)
         done += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -234,7 +285,9 @@ def cpu_baseline_sample(w, inp, budget_s: float) -> dict:
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.threads(),
             "kind": "oracle",
             "sample": f"fp64 oracle forward+backward of {done} of {w.B * w.H} (batch, head) "
-                      f"pairs of the {w.name} workload in {dt:.1f} s (nominal FLOPs)"}
+                      f"pairs of the {w.name} workload"
+                      + (f" with dropout p={dropout_p}" if dropout_p else "")
+                      + f" in {dt:.1f} s (nominal FLOPs)"}
 
 
 def bench_ours(args, rank, world, local_rank):
@@ -249,7 +302,8 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = W.WORKLOADS[args.workload]
-    f_fwd, f_bwd, f_step = step_flops(w)
+    mask_np = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
+    f_fwd, f_bwd, f_step = step_flops(w, mask_np)
 
     inp = W.make_inputs(w, seed=rank_seed(rank))
     first = alloc_set(w, inp, dev)
@@ -258,6 +312,13 @@ def bench_ours(args, rank, world, local_rank):
     nsets = max(2, math.ceil(2 * l2 / per_set) + 1)
     sets = [first] + [alloc_set(w, W.make_inputs(w, seed=rank_seed(rank) + i), dev)
                       for i in range(1, nsets)]
+    if mask_np is not None:
+        mask_t = torch.from_numpy(mask_np).to(dev)
+        for st in sets:
+            st["mask"] = mask_t
+    if args.dropout > 0:
+        for i, st in enumerate(sets):
+            st["drop"] = (args.dropout, 1234 + i)
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
@@ -271,11 +332,15 @@ def bench_ours(args, rank, world, local_rank):
     if status != fa.FA_OK:
         raise RuntimeError(f"device status {status} after warm-up")
 
-    # per-kernel events (forward kernel, backward main kernel), one pair per launch
+    # Per-kernel events (forward kernel, backward main kernel) around the launches of
+    # every `stride`-th step of the timed region (about 256 samples): an event between two
+    # kernels stops the next one from starting early, so most steps run without them.
     K = args.steps
+    stride = max(1, K // 256)
+    sampled = list(range(0, K, stride))
     evs = {0: [], 1: []}
     for which in (0, 1):
-        for _ in range(K):
+        for _ in sampled:
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             b.record(stream)
@@ -289,9 +354,15 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     clocks.mark("t0")
     start.record(stream)
+    si = 0
     for i in range(K):
-        fa.fa_set_timing_events(0, *evs[0][i])
-        fa.fa_set_timing_events(1, *evs[1][i])
+        if si < len(sampled) and sampled[si] == i:
+            fa.fa_set_timing_events(0, *evs[0][si])
+            fa.fa_set_timing_events(1, *evs[1][si])
+            si += 1
+        else:
+            fa.fa_set_timing_events(0)
+            fa.fa_set_timing_events(1)
         run_step(w, sets[i % nsets])
     end.record(stream)
     torch.cuda.synchronize(dev)
@@ -306,8 +377,8 @@ def bench_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {status} after the timed region")
     ms = start.elapsed_time(end)
     max_ms = max_over_ranks(ms, dev if world > 1 else None)
-    k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / K
-    k_bwd = sum(a.elapsed_time(b) for a, b in evs[1]) / K
+    k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / len(evs[0])
+    k_bwd = sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
     value = whole_job_tflops(f_step, world, K, max_ms)
 
     # ---- end to end through the public API with host buffers
@@ -357,11 +428,12 @@ def bench_ours(args, rank, world, local_rank):
                 "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{peak_src} {peak_key}",
                 "flops_per_launch": dom_flops, "launch_ms": dom_ms,
+                "launches_timed": len(evs[0]),
                 "traffic": profile_traffic(dom_name, w.name)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_sample(w, inp, args.cpu_seconds)
+        cpu = cpu_baseline_sample(w, inp, args.cpu_seconds, args.dropout)
 
     per_rank_value = f_step * K / (ms * 1e-3) / 1e12
     line = {
@@ -370,8 +442,10 @@ def bench_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None,
         "dtype": {torch.bfloat16: "bf16", torch.float16: "f16"}[w.dtype],
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
-        "config": {"workload": w.description + ", forward + backward", "B": w.B, "H": w.H,
-                   "N": w.N, "d": w.d, "causal": w.causal,
+        "config": {"workload": w.description + ", forward + backward"
+                   + (", block-sparse local+global pattern" if args.block_sparse else "")
+                   + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
+                   "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "flops_per_step": f_step, "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"{nsets} resident input/output sets ({nsets * per_set / 2**20:.0f} MiB) "
                          "rotated so each step reads data evicted from the 126 MB L2"},
@@ -408,10 +482,17 @@ def bench_reference(args):
     rows_per_step = w.N if total <= 300 else max(16, (w.N * 300) // total)
     rng = np.random.default_rng(0)
 
+    bmask = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
+
     def flops_of(rows, L):
         vis = 0
         for i in rows:
-            vis += min(L, i + 1) if w.causal else L
+            lim = min(L, i + 1) if w.causal else L  # keys < lim pass the causal/padding rule
+            if bmask is None:
+                vis += lim
+            else:
+                for kt in np.nonzero(bmask[i // 128])[0]:
+                    vis += max(0, min(lim, (kt + 1) * 128) - kt * 128)
         return 14.0 * w.d * vis  # 4d forward + 10d backward per visible score
 
     def one(i):
@@ -420,7 +501,8 @@ def bench_reference(args):
         rows = (np.arange(w.N) if rows_per_step >= w.N
                 else np.sort(rng.choice(w.N, rows_per_step, replace=False)))
         oracle.attention_rows(q[b, h], k[b, h], v[b, h], do[b, h], scale=w.scale,
-                              causal=w.causal, kv_len=L, rows=rows)
+                              causal=w.causal, kv_len=L, rows=rows, dropout_p=args.dropout,
+                              seed=1234, bh=b * w.H + h, block_mask=bmask, block_size=128)
         return flops_of(rows, L)
 
     for i in range(args.warmup):
@@ -438,7 +520,10 @@ def bench_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
-        "config": {"workload": w.description + ", forward + backward", "B": w.B, "H": w.H,
+        "config": {"workload": w.description + ", forward + backward"
+                   + (", block-sparse local+global pattern" if args.block_sparse else "")
+                   + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
+                   "B": w.B, "H": w.H,
                    "N": w.N, "d": w.d, "causal": w.causal},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
@@ -458,7 +543,16 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block-sparse", action="store_true",
+                    help="measure the block-sparse path with a local+global block pattern "
+                         "(FLOPs counted over the visible pairs only)")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="measure the dropout path with this drop probability")
     args = ap.parse_args(argv)
+    if args.dropout and args.block_sparse:
+        ap.error("--dropout and --block-sparse measure different paths; pick one")
+    if not (0.0 <= args.dropout < 255.5 / 256):
+        ap.error("--dropout must lie in [0, 255.5/256)")
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local_rank = dist_env()

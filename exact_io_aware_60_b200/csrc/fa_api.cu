@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "fa.h"
 #include "fa_fwd.cuh"
@@ -117,6 +118,25 @@ int check_common(int B, int H, int N, int d, float scale, int dtype) {
     return FA_OK;
 }
 
+// Launches `kern` on `st` with programmatic stream serialization: the kernel may begin
+// while the previous kernel in the stream finishes; it calls pdl_wait() before it reads
+// anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <typename K>
 cudaError_t set_smem(K kern, int bytes, std::atomic<int> *done, int dev) {
     if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
@@ -125,10 +145,10 @@ cudaError_t set_smem(K kern, int bytes, std::atomic<int> *done, int dev) {
     return e;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
                int N, float scale, int causal, const int *kv_len, const uint8_t *bmask,
-               int mask_per_head, cudaStream_t st, int dev) {
+               int mask_per_head, const fa::DropoutParams &drop, cudaStream_t st, int dev) {
     using C = fa::FwdCfg<D>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -151,7 +171,8 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.num_q_tiles = (N + C::BM - 1) / C::BM;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
-    auto kern = fa::fa_fwd_kernel<D, BF16>;
+    p.drop = drop;
+    auto kern = fa::fa_fwd_kernel<D, BF16, DROP>;
     static std::atomic<int> smem_done[kMaxDevices];
     cudaError_t e = set_smem(kern, C::SMEM, smem_done, dev);
     if (e != cudaSuccess) {
@@ -161,8 +182,8 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     const long long grid = (long long)p.num_q_tiles * bh;
     if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
     timing_mark(0, 0, st);
-    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mo, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     timing_mark(0, 1, st);
     if (e != cudaSuccess) {
         record_cuda_error(e, "fa_fwd launch");
@@ -201,11 +222,11 @@ int grid_for(long long work, int threads) {
     return (int)g;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
                const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, float scale,
                int causal, const int *kv_len, const uint8_t *bmask, int mask_per_head,
-               void *workspace, cudaStream_t st, int dev) {
+               const fa::DropoutParams &drop, void *workspace, cudaStream_t st, int dev) {
     using C = fa::BwdCfg<D>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -233,12 +254,14 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     pp.dvec = ws.dvec;
     pp.dq_acc = reinterpret_cast<float4 *>(ws.dq_acc);
     pp.dq_acc_vec4 = bh * (long long)N * D / 4;
+    pp.dscale = DROP ? 1.f / drop.keep_scale : 1.f;
     pp.N = N;
     pp.Npad = num_tiles * 128;
     pp.BH = bh;
     const long long prep_work = std::max(pp.dq_acc_vec4, bh * pp.Npad * (D / 8));
-    fa::fa_bwd_prep_kernel<D, BF16><<<grid_for(prep_work, 256), 256, 0, st>>>(pp);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(fa::fa_bwd_prep_kernel<D, BF16>, dim3(grid_for(prep_work, 256)),
+                               dim3(256), 0, st, pp);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         record_cuda_error(e, "fa_bwd prep launch");
         return FA_ERR_CUDA;
@@ -260,7 +283,10 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
-    auto kern = fa::fa_bwd_kernel<D, BF16>;
+    p.drop = drop;
+    p.dv_mul = drop.keep_scale;
+    p.dk_mul = scale * drop.keep_scale;
+    auto kern = fa::fa_bwd_kernel<D, BF16, DROP>;
     static std::atomic<int> smem_done[kMaxDevices];
     e = set_smem(kern, C::SMEM, smem_done, dev);
     if (e != cudaSuccess) {
@@ -270,8 +296,9 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     const long long grid = (long long)num_tiles * bh;
     if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
     timing_mark(1, 0, st);
-    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mdo,
+                   mdk, mdv, mdq, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     timing_mark(1, 1, st);
     if (e != cudaSuccess) {
         record_cuda_error(e, "fa_bwd launch");
@@ -280,9 +307,10 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 
     // 3. dQ = scale * dQ_acc in the input dtype
     const long long nv4 = bh * (long long)N * D / 4;
-    fa::fa_bwd_convert_kernel<BF16><<<grid_for(nv4, 256), 256, 0, st>>>(
-        reinterpret_cast<const float4 *>(ws.dq_acc), reinterpret_cast<uint2 *>(dq), nv4, scale);
-    e = cudaGetLastError();
+    e = launch_pdl(fa::fa_bwd_convert_kernel<BF16>, dim3(grid_for(nv4, 256)), dim3(256), 0, st,
+                   reinterpret_cast<const float4 *>(ws.dq_acc), reinterpret_cast<uint2 *>(dq), nv4,
+                   DROP ? scale * drop.keep_scale : scale);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         record_cuda_error(e, "fa_bwd convert launch");
         return FA_ERR_CUDA;
@@ -312,6 +340,24 @@ int noalloc_scratch(int dev, void **out) {
     return FA_OK;
 }
 
+// Dropout parameters of probability p_drop: the byte threshold t = rint(256 p) must lie
+// in [0, 255].  Returns false for a p outside that range or not finite.
+bool make_dropout(float p_drop, unsigned long long seed, unsigned int offset,
+                  fa::DropoutParams *dp) {
+    if (!std::isfinite(p_drop) || p_drop < 0.f) return false;
+    const float tf = rintf(p_drop * 256.f);
+    if (tf > 255.f) return false;
+    const uint32_t t = (uint32_t)tf;
+    dp->add16 = (0x8000u - t) * 0x00010001u;
+    dp->seed_lo = (uint32_t)(seed & 0xFFFFFFFFull);
+    dp->seed_hi = (uint32_t)(seed >> 32);
+    dp->offset = offset;
+    dp->keep_scale = 256.f / (float)(256u - t);
+    return true;
+}
+
+const fa::DropoutParams kNoDropout = {0x8000u * 0x00010001u, 0u, 0u, 0u, 1.f};
+
 }  // namespace
 
 extern "C" {
@@ -340,9 +386,11 @@ const char *fa_strerror(int status) {
 
 const char *fa_last_cuda_error(void) { return t_last_error; }
 
+
 static int fwd_common(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                       int H, int N, int d, float scale, int causal, const int *kv_len,
-                      const uint8_t *bmask, int mask_per_head, int dtype, void *stream) {
+                      const uint8_t *bmask, int mask_per_head, const fa::DropoutParams *drop,
+                      int dtype, void *stream) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_INVALID_ARG;
@@ -354,17 +402,26 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, floa
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
-#define FA_FWD_ARGS q, k, v, o, lse, B, H, N, scale, causal, kv_len, bmask, mask_per_head, st, dev
+#define FA_FWD_ARGS q, k, v, o, lse, B, H, N, scale, causal, kv_len, bmask, mask_per_head
+    if (drop) {
+        if (d == 64)
+            return bf16 ? launch_fwd<64, true, true>(FA_FWD_ARGS, *drop, st, dev)
+                        : launch_fwd<64, false, true>(FA_FWD_ARGS, *drop, st, dev);
+        return bf16 ? launch_fwd<128, true, true>(FA_FWD_ARGS, *drop, st, dev)
+                    : launch_fwd<128, false, true>(FA_FWD_ARGS, *drop, st, dev);
+    }
     if (d == 64)
-        return bf16 ? launch_fwd<64, true>(FA_FWD_ARGS) : launch_fwd<64, false>(FA_FWD_ARGS);
-    return bf16 ? launch_fwd<128, true>(FA_FWD_ARGS) : launch_fwd<128, false>(FA_FWD_ARGS);
+        return bf16 ? launch_fwd<64, true, false>(FA_FWD_ARGS, kNoDropout, st, dev)
+                    : launch_fwd<64, false, false>(FA_FWD_ARGS, kNoDropout, st, dev);
+    return bf16 ? launch_fwd<128, true, false>(FA_FWD_ARGS, kNoDropout, st, dev)
+                : launch_fwd<128, false, false>(FA_FWD_ARGS, kNoDropout, st, dev);
 #undef FA_FWD_ARGS
 }
 
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
            int d, float scale, int causal, const int *kv_len, int dtype, void *stream) {
-    return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, nullptr, 0, dtype,
-                      stream);
+    return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, nullptr, 0, nullptr,
+                      dtype, stream);
 }
 
 int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse, int B,
@@ -373,7 +430,16 @@ int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, flo
                        void *stream) {
     if (!block_mask || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
     return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, block_mask,
-                      mask_per_head, dtype, stream);
+                      mask_per_head, nullptr, dtype, stream);
+}
+
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                   int H, int N, int d, float scale, int causal, const int *kv_len, float p_drop,
+                   unsigned long long seed, unsigned int offset, int dtype, void *stream) {
+    fa::DropoutParams dp;
+    if (!make_dropout(p_drop, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+    return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, nullptr, 0, &dp, dtype,
+                      stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -384,8 +450,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 static int bwd_common(const void *q, const void *k, const void *v, const void *o,
                       const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
                       int H, int N, int d, float scale, int causal, const int *kv_len,
-                      const uint8_t *bmask, int mask_per_head, int dtype, void *workspace,
-                      size_t workspace_bytes, void *stream) {
+                      const uint8_t *bmask, int mask_per_head, const fa::DropoutParams *drop,
+                      int dtype, void *workspace, size_t workspace_bytes, void *stream) {
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
         return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
@@ -401,10 +467,19 @@ static int bwd_common(const void *q, const void *k, const void *v, const void *o
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
-#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, bmask, mask_per_head, workspace, st, dev
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, bmask, mask_per_head
+    if (drop) {
+        if (d == 64)
+            return bf16 ? launch_bwd<64, true, true>(FA_BWD_ARGS, *drop, workspace, st, dev)
+                        : launch_bwd<64, false, true>(FA_BWD_ARGS, *drop, workspace, st, dev);
+        return bf16 ? launch_bwd<128, true, true>(FA_BWD_ARGS, *drop, workspace, st, dev)
+                    : launch_bwd<128, false, true>(FA_BWD_ARGS, *drop, workspace, st, dev);
+    }
     if (d == 64)
-        return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
-    return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
+        return bf16 ? launch_bwd<64, true, false>(FA_BWD_ARGS, kNoDropout, workspace, st, dev)
+                    : launch_bwd<64, false, false>(FA_BWD_ARGS, kNoDropout, workspace, st, dev);
+    return bf16 ? launch_bwd<128, true, false>(FA_BWD_ARGS, kNoDropout, workspace, st, dev)
+                : launch_bwd<128, false, false>(FA_BWD_ARGS, kNoDropout, workspace, st, dev);
 #undef FA_BWD_ARGS
 }
 
@@ -413,7 +488,39 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
            float scale, int causal, const int *kv_len, int dtype, void *workspace,
            size_t workspace_bytes, void *stream) {
     return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, kv_len,
-                      nullptr, 0, dtype, workspace, workspace_bytes, stream);
+                      nullptr, 0, nullptr, dtype, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                   const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+                   float scale, int causal, const int *kv_len, float p_drop,
+                   unsigned long long seed, unsigned int offset, int dtype, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    fa::DropoutParams dp;
+    if (!make_dropout(p_drop, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+    return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, kv_len,
+                      nullptr, 0, &dp, dtype, workspace, workspace_bytes, stream);
+}
+
+int fa_dropout_mask(int B, int H, int N, float p_drop, unsigned long long seed,
+                    unsigned int offset, unsigned char *keep, void *stream) {
+    if (!keep || B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    fa::DropoutParams dp;
+    if (!make_dropout(p_drop, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+    const long long bh = (long long)B * H;
+    if ((double)bh * N * N > (double)FA_MAX_ELEMENTS) return FA_ERR_INVALID_ARG;
+    int dev = 0;
+    int rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    const long long work = bh * N * ((N + 15) / 16);
+    fa::dropout_mask_kernel<<<grid_for(work, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        keep, bh, N, dp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "fa_dropout_mask launch");
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
 }
 
 int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
@@ -423,7 +530,7 @@ int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *
                        void *workspace, size_t workspace_bytes, void *stream) {
     if (!block_mask || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
     return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, kv_len,
-                      block_mask, mask_per_head, dtype, workspace, workspace_bytes, stream);
+                      block_mask, mask_per_head, nullptr, dtype, workspace, workspace_bytes, stream);
 }
 
 int fa_selftest_wait_timeout(int limit_us, void *stream) {
@@ -460,10 +567,12 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, c
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
-#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, nullptr, 0, workspace, st, dev
+#define FA_BWD_ARGS q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, causal, kv_len, nullptr, 0, kNoDropout, workspace, st, dev
     if (d == 64)
-        return bf16 ? launch_bwd<64, true>(FA_BWD_ARGS) : launch_bwd<64, false>(FA_BWD_ARGS);
-    return bf16 ? launch_bwd<128, true>(FA_BWD_ARGS) : launch_bwd<128, false>(FA_BWD_ARGS);
+        return bf16 ? launch_bwd<64, true, false>(FA_BWD_ARGS)
+                    : launch_bwd<64, false, false>(FA_BWD_ARGS);
+    return bf16 ? launch_bwd<128, true, false>(FA_BWD_ARGS)
+                : launch_bwd<128, false, false>(FA_BWD_ARGS);
 #undef FA_BWD_ARGS
 }
 

@@ -30,6 +30,7 @@
 
 #include <cuda.h>
 
+#include "dropout.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -46,6 +47,7 @@ struct BwdPrepParams {
     float *dvec;   // [BH][Npad]
     float4 *dq_acc;
     long long dq_acc_vec4;  // number of float4 in dq_acc
+    float dscale;           // D is stored times this (1, or 1 / keep_scale with dropout)
     int N;
     int Npad;
     long long BH;
@@ -58,6 +60,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p) {
     constexpr int G = D / 8;           // threads per row
     constexpr int RPW = 32 / G;        // rows per warp step
+    pdl_wait();
+    pdl_launch_dependents();
     const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long nthreads = (long long)gridDim.x * blockDim.x;
     for (long long i = tid; i < p.dq_acc_vec4; i += nthreads)
@@ -96,7 +100,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
 #pragma unroll
         for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (g == 0 && rr < rows_total) {
-            p.dvec[rr] = acc;
+            p.dvec[rr] = acc * p.dscale;
             p.lse2[rr] = l2;
         }
     }
@@ -107,6 +111,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
 template <bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_convert_kernel(const float4 *acc, uint2 *out,
                                                              long long n_vec4, float scale) {
+    pdl_wait();
+    pdl_launch_dependents();
     const long long nthreads = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec4; i += nthreads) {
         const float4 a = acc[i];
@@ -133,6 +139,11 @@ struct BwdParams {
     float scale;
     float scale_log2;
     int causal;
+    // Dropout variant only: the mask generator, and the epilogue multipliers of dV
+    // (keep_scale) and dK (scale * keep_scale).
+    DropoutParams drop;
+    float dv_mul;
+    float dk_mul;
 };
 
 template <int D>
@@ -189,7 +200,11 @@ struct BwdBars {
     uint32_t tmem_base;
 };
 
-template <int D, bool BF16>
+// DROP: dropout.  With K the keep mask and r = keep_scale, the chain rule gives
+//   dV = r (P o K)^T dO,  dP = r K o (dO V^T),  D = rowsum(dO o O),  dS = P o (dP - D);
+// the kernel computes dS' = P o (K o (dO V^T) - D / r) (D / r comes from the preprocess)
+// and folds r into the dV, dK and dQ output multipliers.
+template <int D, bool BF16, bool DROP>
 __global__ void __launch_bounds__(448, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -269,6 +284,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    pdl_wait();  // the preprocess kernel's outputs are visible from here on
 
     if (warp == C::W_TMA) {
         // ------------------------------ TMA producer ------------------------------
@@ -462,6 +478,25 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
             const int s = i % C::QS;
+            // Dropout keep bits of this key row against queries 64h .. 64h + 63 of tile qi:
+            // bit m of kb[u] = query 32u + 2m, bit m + 16 = query 32u + 2m + 1.  Each lane
+            // of a half-warp draws the Philox blocks of two queries for the half-warp's
+            // 16-key group; a bit transpose hands every lane its own key's bits.
+            uint32_t kb[2] = {0u, 0u};
+            if constexpr (DROP) {
+                const uint32_t grp = (uint32_t)(kt * 128 + quarter * 32 + (lane & 16)) >> 4;
+                const uint32_t q0 = (uint32_t)(qi * 128 + h * 64 + 2 * (lane & 15));
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t a = keep_bits16(
+                        philox4x32_10(grp, q0 + 32 * u, (uint32_t)bh, p.drop.offset, p.drop.seed_lo,
+                                      p.drop.seed_hi), p.drop.add16);
+                    const uint32_t c = keep_bits16(
+                        philox4x32_10(grp, q0 + 32 * u + 1, (uint32_t)bh, p.drop.offset,
+                                      p.drop.seed_lo, p.drop.seed_hi), p.drop.add16);
+                    kb[u] = transpose16x16_halfwarp(a | (c << 16), lane);
+                }
+            }
             if (!mbar_wait(&bars->s_full, i & 1) || !mbar_wait(&bars->q_full[s], (i / C::QS) & 1)) {
                 ok = false;
                 break;
@@ -515,7 +550,18 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 ok = false;
                 break;
             }
-            tmem_st32(tmem + lane_base + C::COL_P + h * C::P_HALF_STRIDE, Pw);
+            if constexpr (DROP) {
+                // the dV operand is P o K; Pw (unmasked) stays for dS
+                uint32_t Pm[32];
+#pragma unroll
+                for (int pi = 0; pi < 32; ++pi) {
+                    const uint32_t x = kb[pi >> 4] << (15 - (pi & 15));
+                    Pm[pi] = Pw[pi] & prmt(x, 0u, 0xBB99u);
+                }
+                tmem_st32(tmem + lane_base + C::COL_P + h * C::P_HALF_STRIDE, Pm);
+            } else {
+                tmem_st32(tmem + lane_base + C::COL_P + h * C::P_HALF_STRIDE, Pw);
+            }
             tc_fence_before();
             mbar_arrive(&bars->p_full);
 
@@ -536,8 +582,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int k = 0; k < 32; k += 2) {
                     const float2 d2 = *reinterpret_cast<const float2 *>(dv + cc * 32 + k);
                     const float2 pp = unpack2<BF16>(Pw[cc * 16 + (k >> 1)]);
-                    const float ds0 = pp.x * (__uint_as_float(w[k]) - d2.x);
-                    const float ds1 = pp.y * (__uint_as_float(w[k + 1]) - d2.y);
+                    float dp0 = __uint_as_float(w[k]);
+                    float dp1 = __uint_as_float(w[k + 1]);
+                    if constexpr (DROP) {
+                        if (!((kb[cc] >> (k >> 1)) & 1u)) dp0 = 0.f;
+                        if (!((kb[cc] >> ((k >> 1) + 16)) & 1u)) dp1 = 0.f;
+                    }
+                    const float ds0 = pp.x * (dp0 - d2.x);
+                    const float ds1 = pp.y * (dp1 - d2.y);
                     pk[k >> 1] = pack2<BF16>(ds0, ds1);
                 }
                 // dS^T pairs -> TMEM, over dP^T columns this warp has just read; A operand
@@ -559,6 +611,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
 
         // ------------------------------ epilogue: dK, dV ------------------------------
+        pdl_launch_dependents();
         if (ok && n > 0) {
             ok = mbar_wait(&bars->dkv_full, 0);
             tc_fence_after();
@@ -571,7 +624,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
             const uint32_t col = (which == 0 ? C::COL_DV : C::COL_DK) + h * HCOLS;
-            const float mul = which == 0 ? 1.f : p.scale;
+            float mul = which == 0 ? 1.f : p.scale;
+            if constexpr (DROP) mul = which == 0 ? p.dv_mul : p.dk_mul;
             uint8_t *stage = which == 0 ? stage_v : stage_k;
 #pragma unroll
             for (int c32 = 0; c32 < HCOLS / 32; ++c32) {

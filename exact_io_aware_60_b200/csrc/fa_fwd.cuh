@@ -46,6 +46,7 @@
 
 #include <cuda.h>
 
+#include "dropout.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -64,6 +65,7 @@ struct FwdParams {
     int num_q_tiles;
     float scale_log2;  // scale * log2(e)
     int causal;
+    DropoutParams drop;  // used by the dropout variant only
 };
 
 template <int D>
@@ -113,7 +115,9 @@ struct FwdBars {
     uint32_t tmem_base;
 };
 
-template <int D, bool BF16>
+// DROP: dropout on the probabilities (the mask is regenerated per element from the
+// counter-based generator; the normaliser is the fp32 sum of the undropped values).
+template <int D, bool BF16, bool DROP>
 __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -192,6 +196,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    pdl_wait();  // inputs written by the previous kernel are visible from here on
 
     if (warp == 4) {
         // ------------------------------ TMA producer ------------------------------
@@ -332,6 +337,24 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 sum1 += p1;
                 pk[c >> 1] = pack2<BF16>(p0, p1);
             }
+            if constexpr (DROP) {
+                // Keys j*BN + 16u .. +15 of this row: one Philox block each; dropped
+                // probabilities become 0 in the operand of the PV product.
+                const uint32_t g0 = (uint32_t)(j * BN) >> 4;
+#pragma unroll
+                for (int u = 0; u < BN / 16; ++u) {
+                    const uint4 r = philox4x32_10(g0 + u, (uint32_t)row, (uint32_t)bh,
+                                                  p.drop.offset, p.drop.seed_lo, p.drop.seed_hi);
+                    const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t m01, m23;
+                        pair_masks(w4[k], p.drop.add16, m01, m23);
+                        pk[8 * u + 2 * k] &= m01;
+                        pk[8 * u + 2 * k + 1] &= m23;
+                    }
+                }
+            }
             l = l * alpha + (sum0 + sum1);
             // Every phase of o_full is waited on, in order, so that a parity wait can
             // never alias a phase two ahead.  P_{j-1} V_{j-1} was issued a whole softmax
@@ -375,6 +398,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
 
         // ------------------------------ epilogue ------------------------------
+        pdl_launch_dependents();
         if (ok && jj > 0) {
             ok = mbar_wait(&bars->o_full, (jj - 1) & 1);
             tc_fence_after();
@@ -386,7 +410,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tmem_ld16(ob + D, r);
             l_round = __uint_as_float(r[0]);
         }
-        const float inv = (l > 0.f && l_round > 0.f) ? 1.f / l_round : 0.f;
+        // Without dropout the output is divided by the sum of the rounded probabilities
+        // the MMA used; with dropout those no longer sum the row, and the output is
+        // (sum of kept P v) * keep_scale / l.
+        float inv;
+        if constexpr (DROP) inv = (l > 0.f) ? p.drop.keep_scale / l : 0.f;
+        else inv = (l > 0.f && l_round > 0.f) ? 1.f / l_round : 0.f;
 #pragma unroll
         for (int hf = 0; hf < C::HALVES; ++hf) {
             uint32_t w[32];

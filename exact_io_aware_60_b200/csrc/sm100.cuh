@@ -99,6 +99,15 @@ __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
     }
 }
 
+// Programmatic dependent launch: kernels of one step are launched so that the next one
+// may start early.  pdl_wait() blocks until the previous kernel in the stream has
+// completed and its memory is visible (it returns at once if there is no such
+// dependency); pdl_launch_dependents() lets the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier over `count` threads (a multiple of 32) of this CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

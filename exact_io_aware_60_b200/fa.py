@@ -77,6 +77,15 @@ def lib():
             L.fa_bwd_blocksparse.restype = i
             L.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f,
                                              i, vp, vp, i, i, vp, sz, vp]
+            u64, u32 = ctypes.c_ulonglong, ctypes.c_uint
+            L.fa_fwd_dropout.restype = i
+            L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, f, u64, u32, i,
+                                         vp]
+            L.fa_bwd_dropout.restype = i
+            L.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp,
+                                         f, u64, u32, i, vp, sz, vp]
+            L.fa_dropout_mask.restype = i
+            L.fa_dropout_mask.argtypes = [i, i, i, f, u64, u32, vp, vp]
             L.fa_bwd_noalloc.restype = i
             L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i,
                                          vp, i, vp]
@@ -236,6 +245,56 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, causal: b
                               _kv_ptr(kv_len, B), _dtype_code(q), _stream_handle(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd_noalloc")
+
+
+def fa_fwd_dropout(q, k, v, o, lse, *, scale: float, p_drop: float, seed: int, offset: int = 0,
+                   causal: bool = False, kv_len=None, stream=None) -> None:
+    """Forward pass with dropout of probability ``p_drop`` on the attention weights; the
+    keep mask is drawn from (``seed``, ``offset``) and never stored (see include/fa.h)."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    rc = lib().fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                              _kv_ptr(kv_len, B), float(p_drop), int(seed), int(offset),
+                              _dtype_code(q), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_dropout")
+
+
+def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, *, scale: float, p_drop: float, seed: int,
+                   offset: int = 0, causal: bool = False, kv_len=None, workspace: torch.Tensor,
+                   stream=None) -> None:
+    """Backward pass of :func:`fa_fwd_dropout`; give it the same p_drop, seed, offset."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        _check(t, name, (B, H, N, d), q.dtype)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise FAError(FA_ERR_INVALID_ARG, "workspace must be a contiguous uint8 CUDA tensor")
+    rc = lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                              _kv_ptr(kv_len, B), float(p_drop), int(seed), int(offset),
+                              _dtype_code(q), workspace.data_ptr(), workspace.numel(),
+                              _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_dropout")
+
+
+def fa_dropout_mask(keep, *, p_drop: float, seed: int, offset: int = 0, stream=None) -> None:
+    """Writes the keep mask of the dropout calls into ``keep``, a uint8 CUDA tensor
+    [B, H, N, N] (1 = kept)."""
+    if not isinstance(keep, torch.Tensor) or not keep.is_cuda or keep.dtype != torch.uint8 \
+            or not keep.is_contiguous() or keep.dim() != 4 or keep.shape[2] != keep.shape[3]:
+        raise FAError(FA_ERR_INVALID_ARG, "keep must be a contiguous uint8 CUDA tensor [B,H,N,N]")
+    B, H, N, _ = keep.shape
+    rc = lib().fa_dropout_mask(B, H, N, float(p_drop), int(seed), int(offset), keep.data_ptr(),
+                               _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_dropout_mask")
 
 
 def fa_set_timing_events(which: int, start=None, stop=None) -> None:

@@ -158,6 +158,51 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, void *stream);
 
 /*
+ * Attention with dropout on the probabilities (promptingindex page, "Why attention is
+ * memory-bound, not compute-bound": dropout is the op between the softmax and the
+ * product with V).  Identical to fa_fwd / fa_bwd except that
+ *     O_i = sum_j P_ij K_ij r v_j,   r = 256 / (256 - t),   t = rint(256 * p_drop),
+ * where P is the softmax of the Mask rule above (LSE is unchanged) and K_ij = 1 when
+ * the random byte of element (i, j) is >= t.  The backward call returns the gradients
+ * of that O (dV = r (P o K)^T dO, dP = r K o (dO V^T), D = rowsum(dO o O), dS = P o
+ * (dP - D)) and must be given the same p_drop, seed and offset as the forward call.
+ * The mask is never stored: both calls regenerate it (the recomputation of NOTE-005,
+ * "Method", applied to the random numbers).
+ *   p_drop : drop probability, used as t / 256 (nearest multiple of 1/256, ties to
+ *            even); t must lie in [0, 255], i.e. 0 <= p_drop < 255.5 / 256.  p_drop = 0
+ *            keeps everything (same O as fa_fwd up to the normaliser's rounding).
+ *   seed   : 64-bit key of the generator.
+ *   offset : 32-bit stream number (e.g. layer or step), fourth word of the counter.
+ * Random byte of element (i, j) of head bh = b * H + h: byte j mod 16 of the 16 output
+ * bytes (byte k = bits 8 (k mod 4) .. +7 of word k / 4) of Philox4x32-10 (Salmon et al.,
+ * "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011) with counter
+ * (j / 16, i, bh, offset) and key (seed mod 2^32, seed >> 32).
+ * Returns FA_ERR_INVALID_ARG for a p_drop outside the range; otherwise as fa_fwd / fa_bwd.
+ */
+FA_API int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int H, int N, int d, float scale, int causal,
+                          const int *kv_len, float p_drop, unsigned long long seed,
+                          unsigned int offset, int dtype, void *stream);
+
+FA_API int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o,
+                          const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                          int B, int H, int N, int d, float scale, int causal,
+                          const int *kv_len, float p_drop, unsigned long long seed,
+                          unsigned int offset, int dtype, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
+ * The keep mask that fa_fwd_dropout / fa_bwd_dropout use, written out:
+ *   keep : DEVICE pointer to uint8 [B * H][N][N], keep[bh][i][j] = K_ij (1 or 0),
+ *          written by the call (asynchronously on `stream`).
+ * For inspection and tests; it materialises N^2 bytes per head, which the attention
+ * calls never do.  Returns FA_ERR_INVALID_ARG for a null pointer, B, H or N < 1, a bad
+ * p_drop, or more than FA_MAX_ELEMENTS mask bytes.
+ */
+FA_API int fa_dropout_mask(int B, int H, int N, float p_drop, unsigned long long seed,
+                           unsigned int offset, unsigned char *keep, void *stream);
+
+/*
  * Backward pass for callers that cannot allocate device memory.  The FlashAttention
  * pages have no counterpart to this entry point: it exists for the environment, not the
  * method.  Some hosts of this library may not call cudaMalloc at all: plugins inside

@@ -124,3 +124,46 @@ def test_blocksparse_rejects_missing_or_bad_mask():
     rc = L.fa_bwd_blocksparse(P, P, P, P, P, P, P, P, P, a["B"], a["H"], a["N"], a["d"],
                               a["scale"], 0, None, None, 0, 0, P * 16, 1 << 30, None)
     assert rc == fa.FA_ERR_INVALID_ARG
+
+
+def call_fwd_dropout(p_drop, **over):
+    a = dict(GOOD, q=P, k=P, v=P, o=P, lse=P, kv=None)
+    a.update(over)
+    return fa.lib().fa_fwd_dropout(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                                   a["N"], a["d"], a["scale"], a["causal"], a["kv"], p_drop,
+                                   1234, 0, a["dtype"], None)
+
+
+def call_bwd_dropout(p_drop, **over):
+    a = dict(GOOD, ws=P, ws_bytes=1 << 30, kv=None)
+    a.update(over)
+    return fa.lib().fa_bwd_dropout(P, P, P, P, P, P, P, P, P, a["B"], a["H"], a["N"], a["d"],
+                                   a["scale"], a["causal"], a["kv"], p_drop, 1234, 0, a["dtype"],
+                                   a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("p_drop", [float("nan"), float("inf"), -0.01, 255.6 / 256, 1.0, 3.0])
+def test_dropout_rejects_bad_probability_on_host(p_drop):
+    assert call_fwd_dropout(p_drop) == fa.FA_ERR_INVALID_ARG
+    assert call_bwd_dropout(p_drop) == fa.FA_ERR_INVALID_ARG
+    assert fa.lib().fa_dropout_mask(1, 1, 16, p_drop, 1, 0, P, None) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(q=None), dict(B=0), dict(scale=-1.0), dict(dtype=5)])
+def test_dropout_forward_keeps_the_common_checks(over):
+    assert call_fwd_dropout(0.1, **over) == fa.FA_ERR_INVALID_ARG
+
+
+def test_dropout_backward_keeps_the_common_checks():
+    assert call_bwd_dropout(0.1, ws_bytes=16) == fa.FA_ERR_INVALID_ARG
+    assert call_bwd_dropout(0.1, ws=P + 16) == fa.FA_ERR_INVALID_ARG
+    assert call_bwd_dropout(0.1, d=96) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_dropout_mask_rejects_bad_arguments_on_host():
+    L = fa.lib()
+    assert L.fa_dropout_mask(1, 1, 16, 0.1, 1, 0, None, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_dropout_mask(0, 1, 16, 0.1, 1, 0, P, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_dropout_mask(1, 1, 0, 0.1, 1, 0, P, None) == fa.FA_ERR_INVALID_ARG
+    # more than FA_MAX_ELEMENTS (2^40) mask bytes
+    assert L.fa_dropout_mask(1 << 10, 1, 1 << 16, 0.1, 1, 0, P, None) == fa.FA_ERR_INVALID_ARG

@@ -92,3 +92,34 @@ def test_profile_traffic_only_for_current_sources(tmp_path, monkeypatch):
     assert bench.profile_traffic("fa_bwd_kernel", "gpt2") == 12345.0
     (csrc / "k.cuh").write_text("kernel v2")
     assert bench.profile_traffic("fa_bwd_kernel", "gpt2") is None
+
+
+def test_visible_pairs_counts():
+    import numpy as np
+    T, N = 8, 1024
+    ones = np.ones((T, T), np.uint8)
+    assert bench.visible_pairs(N, ones, True) == N * (N + 1) // 2
+    assert bench.visible_pairs(N, ones, False) == N * N
+    assert bench.visible_pairs(300, np.ones((3, 3), np.uint8), False) == 300 * 300
+    eye = np.eye(T, dtype=np.uint8)
+    assert bench.visible_pairs(N, eye, False) == T * 128 * 128
+    assert bench.visible_pairs(N, eye, True) == T * 128 * 129 // 2
+
+
+@pytest.mark.parametrize("flags,suffix", [(["--dropout", "0.1"], "dropout p=0.1"),
+                                          (["--block-sparse"], "block-sparse")])
+def test_reference_arm_follows_the_measured_path(flags, suffix):
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3",
+                         "--workload", "tiny"] + flags)
+    assert rc == 0
+    d = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert suffix in d["config"]["workload"] and d["value"] > 0
+
+
+def test_dropout_and_block_sparse_are_exclusive():
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--dropout", "0.1", "--block-sparse"])
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--dropout", "1.0"])
