@@ -71,6 +71,11 @@ def _load():
                 dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_double, ctypes.c_int,
                 ctypes.c_long, ctypes.c_void_p, ctypes.c_long, ctypes.POINTER(_Dropout), lp,
                 ctypes.c_long, dp, dp, dp, dp, dp]
+            lib.oracle_attention_rows_qk.restype = ctypes.c_int
+            lib.oracle_attention_rows_qk.argtypes = [
+                dp, dp, dp, dp, ctypes.c_long, ctypes.c_long, ctypes.c_long, ctypes.c_double,
+                ctypes.c_int, ctypes.c_long, ctypes.c_void_p, ctypes.c_long,
+                ctypes.POINTER(_Dropout), lp, ctypes.c_long, dp, dp, dp, dp, dp]
             u32p = ctypes.POINTER(ctypes.c_uint)
             lib.oracle_philox4x32_10.restype = None
             lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
@@ -144,7 +149,9 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
                    offset=0, bh=0):
     """Exact attention of one (batch, head) for the query rows ``rows``.
 
-    q, k, v, dout: ``[N, d]`` arrays (cast to fp64).  ``kv_len``: valid keys (None = N).
+    q, dout: ``[Nq, d]``; k, v: ``[Nk, d]`` (cast to fp64).  With Nq != Nk the queries are
+    the last Nq positions of the key sequence (causal: key j visible to query i when
+    j <= i + Nk - Nq).  ``kv_len``: valid keys (None = Nk).
     ``block_mask``: optional ``[nb, nb]`` array (nb = ceil(N / block_size)); key j is
     visible to query i only where ``block_mask[i // block_size, j // block_size]`` != 0.
     ``dropout_p``, ``seed``, ``offset``, ``bh``: dropout on the probabilities with the
@@ -153,11 +160,12 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
     and (if ``want_dkdv``) ``dk``, ``dv [N,d]`` summed over the given rows only.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
-    N, d = q.shape
+    Nq, d = q.shape
+    N = k.shape[0]
     assert k.shape == (N, d) and v.shape == (N, d)
     L = N if kv_len is None else int(kv_len)
     if rows is None:
-        rows = np.arange(N, dtype=np.int64)
+        rows = np.arange(Nq, dtype=np.int64)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     R = rows.shape[0]
     o = np.zeros((R, d))
@@ -165,7 +173,7 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
     dq = dk = dv = None
     if dout is not None:
         dout = _f64(dout)
-        assert dout.shape == (N, d)
+        assert dout.shape == (Nq, d)
         dq = np.zeros((R, d))
         if want_dkdv:
             dk = np.zeros((N, d))
@@ -176,8 +184,8 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
         mask_arr = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
         assert mask_arr.shape == (nb, nb), (mask_arr.shape, nb)
     drop = _Dropout(dropout_threshold(dropout_p), int(seed), int(offset), int(bh))
-    rc = _load().oracle_attention_rows_ex(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), N, d, float(scale), int(bool(causal)), L,
+    rc = _load().oracle_attention_rows_qk(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), Nq, N, d, float(scale), int(bool(causal)), L,
         None if mask_arr is None else mask_arr.ctypes.data_as(ctypes.c_void_p),
         int(block_size), ctypes.byref(drop), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)),
         R, _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv))
@@ -194,7 +202,8 @@ def attention_rows(q, k, v, dout=None, *, scale, causal=False, kv_len=None, rows
 
 def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=None,
               block_mask=None, block_size=128, dropout_p=0.0, seed=0, offset=0):
-    """Exact attention over ``[B, H, N, d]`` arrays, one (b, h) at a time.
+    """Exact attention over ``[B, H, N, d]`` arrays, one (b, h) at a time (k, v may be
+    ``[B, H, Nk, d]`` with Nk != N: see ``attention_rows``).
 
     ``kv_len``: per-batch valid key counts (length B) or None.  ``heads``: optional list
     of (b, h) pairs to evaluate; the others are left as NaN in the outputs.
@@ -204,12 +213,14 @@ def attention(q, k, v, dout=None, *, scale, causal=False, kv_len=None, heads=Non
     """
     q = np.asarray(q)
     B, H, N, d = q.shape
+    Nk = np.asarray(k).shape[2]
     o = np.full((B, H, N, d), np.nan)
     lse = np.full((B, H, N), np.nan)
     res = {"o": o, "lse": lse}
     if dout is not None:
-        for name in ("dq", "dk", "dv"):
-            res[name] = np.full((B, H, N, d), np.nan)
+        res["dq"] = np.full((B, H, N, d), np.nan)
+        for name in ("dk", "dv"):
+            res[name] = np.full((B, H, Nk, d), np.nan)
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     for b, h in pairs:
         L = None if kv_len is None else int(kv_len[b])

@@ -34,6 +34,12 @@
  *   dK_j  = scale * sum_i dS_ij q_i
  * A row with no allowed key has O = 0, LSE = -inf, zero gradients.
  *
+ * Queries and keys may differ in number (the inference shape: a short block of Nq new
+ * queries against Nk cached keys, aicassindra page "Inference", stackzen glossary).  The
+ * queries are then the last Nq positions of the key sequence, so the causal rule reads
+ *   allowed(i, j) = (j < L) && (!causal || j <= i + Nk - Nq),
+ * which is the rule above when Nq = Nk.
+ *
  * Block-sparse attention (promptingindex page, "Benchmark results": the same tiling
  * applied to a sparse pattern; NOTE-005, "Key components": the block-sparse extension)
  * restricts the allowed set further: with a block mask M of (ceil(N/bs))^2 bytes,
@@ -132,9 +138,9 @@ int oracle_dropout_keep(unsigned threshold, unsigned long long seed, unsigned of
     return 0;
 }
 
-static int is_allowed(long i, long j, int causal, long L, const block_mask_t *bm)
+static int is_allowed(long i, long j, int causal, long L, long off, const block_mask_t *bm)
 {
-    if (!(j < L && (!causal || j <= i))) return 0;
+    if (!(j < L && (!causal || j <= i + off))) return 0;
     if (bm && bm->m) return bm->m[(i / bm->bs) * bm->nb + (j / bm->bs)] != 0;
     return 1;
 }
@@ -162,19 +168,24 @@ int oracle_threads(void)
 /*
  * Exact attention for the query rows rows[0..R) of one (batch, head).
  *
- * q, k, v, dout : N x d fp64, row-major.  dout may be NULL (forward only).
- * L             : number of valid keys (key padding), 0 <= L <= N.
+ * q, dout       : Nq x d fp64, row-major.  dout may be NULL (forward only).
+ * k, v          : Nk x d fp64, row-major.
+ * L             : number of valid keys (key padding), 0 <= L <= Nk.
  * o             : R x d out; lse : R out (natural log).
  * dq            : R x d out or NULL.
- * dk, dv        : N x d, ACCUMULATED (+=) with the contributions of the given rows, or
- *                 NULL.  Over rows = 0..N-1 they are the full gradients.
+ * dk, dv        : Nk x d, ACCUMULATED (+=) with the contributions of the given rows, or
+ *                 NULL.  Over rows = 0..Nq-1 they are the full gradients.
+ * A block mask or dropout needs Nq = Nk.
  */
-int oracle_attention_rows_ex(const double *q, const double *k, const double *v,
-                             const double *dout, long N, long d, double scale, int causal, long L,
-                             const unsigned char *block_mask, long block_size,
+int oracle_attention_rows_qk(const double *q, const double *k, const double *v,
+                             const double *dout, long Nq, long Nk, long d, double scale,
+                             int causal, long L, const unsigned char *block_mask, long block_size,
                              const oracle_dropout_t *drop, const long *rows, long R, double *o,
                              double *lse, double *dq, double *dk, double *dv)
 {
+    const long N = Nk; /* keys per row of the score matrix */
+    const long off = Nk - Nq;
+    if (Nq < 1 || (Nq != Nk && (block_mask || (drop && drop->threshold > 0)))) return ORACLE_ERR_ARG;
     if (drop && drop->threshold > 255) return ORACLE_ERR_ARG;
     const int dropping = drop && drop->threshold > 0;
     const double keep_scale = dropping ? 256.0 / (256.0 - (double)drop->threshold) : 1.0;
@@ -191,7 +202,7 @@ int oracle_attention_rows_ex(const double *q, const double *k, const double *v,
         return ORACLE_ERR_ARG;
     if ((dq || dk || dv) && !dout) return ORACLE_ERR_ARG;
     for (long r = 0; r < R; ++r)
-        if (rows[r] < 0 || rows[r] >= N) return ORACLE_ERR_ARG;
+        if (rows[r] < 0 || rows[r] >= Nq) return ORACLE_ERR_ARG;
     if (R == 0) return ORACLE_OK;
 
     const long PR = panel_rows(N, R);
@@ -217,7 +228,7 @@ int oracle_attention_rows_ex(const double *q, const double *k, const double *v,
             /* 1. scaled scores with the mask applied */
             double m = -INFINITY;
             for (long j = 0; j < N; ++j) {
-                if (!is_allowed(i, j, causal, L, bm)) {
+                if (!is_allowed(i, j, causal, L, off, bm)) {
                     Srow[j] = -INFINITY;
                     continue;
                 }
@@ -271,7 +282,7 @@ int oracle_attention_rows_ex(const double *q, const double *k, const double *v,
             double *dSrow = dS + r * N;
             double D = 0.0;
             for (long j = 0; j < N; ++j) {
-                if (!is_allowed(i, j, causal, L, bm)) {
+                if (!is_allowed(i, j, causal, L, off, bm)) {
                     dSrow[j] = 0.0;
                     continue;
                 }
@@ -324,6 +335,17 @@ int oracle_attention_rows_ex(const double *q, const double *k, const double *v,
     free(dS);
     free(KR);
     return ORACLE_OK;
+}
+
+/* Nq = Nk = N. */
+int oracle_attention_rows_ex(const double *q, const double *k, const double *v,
+                             const double *dout, long N, long d, double scale, int causal, long L,
+                             const unsigned char *block_mask, long block_size,
+                             const oracle_dropout_t *drop, const long *rows, long R, double *o,
+                             double *lse, double *dq, double *dk, double *dv)
+{
+    return oracle_attention_rows_qk(q, k, v, dout, N, N, d, scale, causal, L, block_mask,
+                                    block_size, drop, rows, R, o, lse, dq, dk, dv);
 }
 
 /* oracle_attention_rows_ex without dropout. */
