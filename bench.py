@@ -66,7 +66,10 @@ def max_over_ranks(value: float, device=None) -> float:
 def step_flops(w, block_mask=None) -> tuple:
     """(forward, backward, total) FLOPs of one step.  Dense: the nominal count.  With a
     block mask: 4 d per visible (query, key) pair forward and 10 d backward (the work the
-    kernels actually do; masked blocks are skipped)."""
+    kernels actually do; masked blocks are skipped).  Inference shape: forward only."""
+    if w.inference:
+        f = w.nominal_flops()[0]
+        return f, 0.0, f
     if block_mask is None:
         f, b = w.nominal_flops()
         return f, b, f + b
@@ -223,9 +226,23 @@ def gpu_pci_id(dev: int) -> str:
 
 # ------------------------------------------------------------------ our arm
 
+def inference_bytes(w) -> float:
+    """Compulsory HBM bytes of one inference forward: read Q, K, V, write O and LSE."""
+    e = 2
+    return float(w.B * w.H * (2 * w.N * w.d * e + 2 * w.n_q * w.d * e + 4 * w.n_q))
+
+
 def alloc_set(w, inp, dev):
     import torch
     from exact_io_aware_60_b200 import fa
+    if w.inference:
+        s = {n: inp[n].to(dev) for n in ("q", "k", "v")}
+        s["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
+        s["o"] = torch.empty_like(s["q"])
+        s["lse"] = torch.empty(s["q"].shape[:-1], dtype=torch.float32, device=dev)
+        n = fa.fa_fwd_splitkv_workspace_bytes(w.B, w.H, w.n_q, w.N, w.d, 0)
+        s["ws_split"] = torch.empty(n, dtype=torch.uint8, device=dev) if n > 0 else None
+        return s
     s = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
     s["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
     s["o"] = torch.empty_like(s["q"])
@@ -241,6 +258,11 @@ def set_bytes(s) -> int:
 
 def run_step(w, s, stream=None):
     from exact_io_aware_60_b200 import fa
+    if w.inference:
+        fa.fa_fwd_splitkv(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale,
+                          causal=w.causal, kv_len=s["kv_len"], num_splits=0,
+                          workspace=s["ws_split"], stream=stream)
+        return
     if s.get("drop") is not None:
         p, seed = s["drop"]
         fa.fa_fwd_dropout(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale, p_drop=p,
@@ -267,14 +289,16 @@ def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0) -> dict
     """The oracle (as it stands) on whole heads of the workload until ``budget_s`` of CPU
     time has passed (at least one head)."""
     import oracle
-    q, k, v, do = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+    do = None if w.inference else inp["do"].double().numpy()
     kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     t0 = time.perf_counter()
     done = 0
     for b, h in heads:
         L = w.N if kv is None else int(kv[b])
-        oracle.attention_rows(q[b, h], k[b, h], v[b, h], do[b, h], scale=w.scale,
+        oracle.attention_rows(q[b, h], k[b, h], v[b, h], None if do is None else do[b, h],
+                              scale=w.scale,
                               causal=w.causal, kv_len=L, dropout_p=dropout_p, seed=1234,
                               bh=b * w.H + h)
         done += 1
@@ -284,7 +308,8 @@ def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0) -> dict
     flops = step_flops(w)[2] * done / (w.B * w.H)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": f"fp64 oracle forward+backward of {done} of {w.B * w.H} (batch, head) "
+            "sample": f"fp64 oracle {'forward' if w.inference else 'forward+backward'} of "
+                      f"{done} of {w.B * w.H} (batch, head) "
                       f"pairs of the {w.name} workload"
                       + (f" with dropout p={dropout_p}" if dropout_p else "")
                       + f" in {dt:.1f} s (nominal FLOPs)"}
@@ -378,23 +403,25 @@ def bench_ours(args, rank, world, local_rank):
     ms = start.elapsed_time(end)
     max_ms = max_over_ranks(ms, dev if world > 1 else None)
     k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / len(evs[0])
-    k_bwd = sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
+    k_bwd = 0.0 if w.inference else sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
     value = whole_job_tflops(f_step, world, K, max_ms)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
+        in_names = ("q", "k", "v") if w.inference else ("q", "k", "v", "do")
+        out_names = ("o", "lse") if w.inference else ("o", "lse", "dq", "dk", "dv")
+        host = {n: inp[n].pin_memory() for n in in_names}
         outs = {n: torch.empty(first[n].shape, dtype=first[n].dtype, pin_memory=True)
-                for n in ("o", "lse", "dq", "dk", "dv")}
+                for n in out_names}
         Ke = max(3, min(K, args.e2e_steps))
         s = first
 
         def e2e_step():
-            for n in ("q", "k", "v", "do"):
+            for n in in_names:
                 s[n].copy_(host[n], non_blocking=True)
             run_step(w, s)
-            for n in ("o", "lse", "dq", "dk", "dv"):
+            for n in out_names:
                 outs[n].copy_(s[n], non_blocking=True)
 
         for _ in range(2):
@@ -430,6 +457,13 @@ def bench_ours(args, rank, world, local_rank):
                 "flops_per_launch": dom_flops, "launch_ms": dom_ms,
                 "launches_timed": len(evs[0]),
                 "traffic": profile_traffic(dom_name, w.name)}
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    if w.inference and f_fwd / inference_bytes(w) < peak * 1e3 / hbm:
+        # below the ridge point: the split-KV forward is bound by streaming K and V
+        gbs = inference_bytes(w) / (dom_ms * 1e-3) / 1e9
+        roofline.update({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                         "bytes_per_launch": inference_bytes(w), "tflops": achieved})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -442,19 +476,24 @@ def bench_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None,
         "dtype": {torch.bfloat16: "bf16", torch.float16: "f16"}[w.dtype],
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
-        "config": {"workload": w.description + ", forward + backward"
+        "config": {"workload": w.description
+                   + (", inference forward (split-KV)" if w.inference else ", forward + backward")
                    + (", block-sparse local+global pattern" if args.block_sparse else "")
                    + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
                    "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   **({"Nq": w.n_q} if w.inference else {}),
                    "flops_per_step": f_step, "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"{nsets} resident input/output sets ({nsets * per_set / 2**20:.0f} MiB) "
                          "rotated so each step reads data evicted from the 126 MB L2"},
         "pct_of_peak": 100.0 * per_rank_value / peak,
-        "kernels": {"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12},
-                    "fa_bwd_kernel": {"ms": k_bwd, "tflops": f_bwd / (k_bwd * 1e-3) / 1e12}},
+        "kernels": ({"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12}}
+                    if w.inference else
+                    {"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12},
+                     "fa_bwd_kernel": {"ms": k_bwd, "tflops": f_bwd / (k_bwd * 1e-3) / 1e12}}),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": 4 * K,
+        "gpu_launches": ((1 + int(first.get("ws_split") is not None)) * K if w.inference
+                         else 4 * K),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
@@ -475,32 +514,37 @@ def bench_reference(args):
     from exact_io_aware_60_b200 import workloads as W
     w = W.WORKLOADS[args.workload]
     inp = W.make_inputs(w, seed=0)
-    q, k, v, do = (inp[n].double().numpy() for n in ("q", "k", "v", "do"))
+    q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+    do = None if w.inference else inp["do"].double().numpy()
     kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     total = args.steps + args.warmup
-    rows_per_step = w.N if total <= 300 else max(16, (w.N * 300) // total)
+    nq = w.n_q
+    rows_per_step = nq if total <= 300 else max(min(16, nq), (nq * 300) // total)
     rng = np.random.default_rng(0)
+    off = w.N - nq  # inference shape: queries are the last nq positions
 
     bmask = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
 
     def flops_of(rows, L):
         vis = 0
         for i in rows:
-            lim = min(L, i + 1) if w.causal else L  # keys < lim pass the causal/padding rule
+            lim = min(L, i + 1 + off) if w.causal else L  # keys < lim pass causal/padding
             if bmask is None:
                 vis += lim
             else:
                 for kt in np.nonzero(bmask[i // 128])[0]:
                     vis += max(0, min(lim, (kt + 1) * 128) - kt * 128)
-        return 14.0 * w.d * vis  # 4d forward + 10d backward per visible score
+        # 4d forward (+ 10d backward) per visible score
+        return (4.0 if w.inference else 14.0) * w.d * vis
 
     def one(i):
         b, h = heads[i % len(heads)]
         L = w.N if kv is None else int(kv[b])
-        rows = (np.arange(w.N) if rows_per_step >= w.N
-                else np.sort(rng.choice(w.N, rows_per_step, replace=False)))
-        oracle.attention_rows(q[b, h], k[b, h], v[b, h], do[b, h], scale=w.scale,
+        rows = (np.arange(nq) if rows_per_step >= nq
+                else np.sort(rng.choice(nq, rows_per_step, replace=False)))
+        oracle.attention_rows(q[b, h], k[b, h], v[b, h], None if do is None else do[b, h],
+                              scale=w.scale,
                               causal=w.causal, kv_len=L, rows=rows, dropout_p=args.dropout,
                               seed=1234, bh=b * w.H + h, block_mask=bmask, block_size=128)
         return flops_of(rows, L)
@@ -513,18 +557,20 @@ def bench_reference(args):
         fl += one(args.warmup + i)
     dt = time.perf_counter() - t0
     value = fl / dt / 1e12
-    sample = (f"fp64 oracle forward+backward of {rows_per_step} query rows of one (batch, head) "
-              f"pair per step, {w.name} workload")
+    sample = (f"fp64 oracle {'forward' if w.inference else 'forward+backward'} of "
+              f"{rows_per_step} query rows of one (batch, head) pair per step, {w.name} workload")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
-        "config": {"workload": w.description + ", forward + backward"
+        "config": {"workload": w.description
+                   + (", inference forward (split-KV)" if w.inference else ", forward + backward")
                    + (", block-sparse local+global pattern" if args.block_sparse else "")
                    + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
                    "B": w.B, "H": w.H,
-                   "N": w.N, "d": w.d, "causal": w.causal},
+                   "N": w.N, "d": w.d, "causal": w.causal,
+                   **({"Nq": w.n_q} if w.inference else {})},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

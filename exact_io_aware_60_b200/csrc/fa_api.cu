@@ -145,23 +145,39 @@ cudaError_t set_smem(K kern, int bytes, std::atomic<int> *done, int dev) {
     return e;
 }
 
-template <int D, bool BF16, bool DROP>
+// Split-KV output of one launch: fp32 partial outputs and LSEs (see FwdParams).
+struct SplitOut {
+    float *part_o = nullptr;
+    float *part_lse = nullptr;
+    int num_splits = 1;
+    int blocks_per_split = 0;
+};
+
+template <int D, bool BF16, bool DROP, bool SPLIT>
 int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
-               int N, float scale, int causal, const int *kv_len, const uint8_t *bmask,
-               int mask_per_head, const fa::DropoutParams &drop, cudaStream_t st, int dev) {
+               int N, int Nk, float scale, int causal, const int *kv_len, const uint8_t *bmask,
+               int mask_per_head, const fa::DropoutParams &drop, const SplitOut &so,
+               cudaStream_t st, int dev) {
     using C = fa::FwdCfg<D>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const long long bh = (long long)B * H;
     CUtensorMap mq, mk, mv, mo;
+    // (in split mode O is written by the combine kernel; the O map is then unused but valid)
     if (!make_map(&mq, q, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, k, dt, 2, D, N, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, v, dt, 2, D, N, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, k, dt, 2, D, Nk, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, v, dt, 2, D, Nk, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mo, o, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return FA_ERR_CUDA;
     fa::FwdParams p;
     p.lse = lse;
     p.kv_len = kv_len;
+    p.part_o = so.part_o;
+    p.part_lse = so.part_lse;
+    p.num_splits = so.num_splits;
+    p.kv_blocks_per_split = so.blocks_per_split;
+    p.Nk = Nk;
+    p.causal_off = Nk - N;
     p.bmask = bmask;
     p.bmask_T = (N + 127) / 128;
     p.bmask_bh_stride = mask_per_head ? (long long)p.bmask_T * p.bmask_T : 0;
@@ -172,14 +188,14 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.drop = drop;
-    auto kern = fa::fa_fwd_kernel<D, BF16, DROP>;
+    auto kern = fa::fa_fwd_kernel<D, BF16, DROP, SPLIT>;
     static std::atomic<int> smem_done[kMaxDevices];
     cudaError_t e = set_smem(kern, C::SMEM, smem_done, dev);
     if (e != cudaSuccess) {
         record_cuda_error(e, "cudaFuncSetAttribute(fwd)");
         return FA_ERR_CUDA;
     }
-    const long long grid = (long long)p.num_q_tiles * bh;
+    const long long grid = (long long)p.num_q_tiles * so.num_splits * bh;
     if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
     timing_mark(0, 0, st);
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mo, p);
@@ -358,6 +374,72 @@ bool make_dropout(float p_drop, unsigned long long seed, unsigned int offset,
 
 const fa::DropoutParams kNoDropout = {0x8000u * 0x00010001u, 0u, 0u, 0u, 1.f};
 
+// Key splits of the split-KV forward: `requested` (> 0) capped by the key blocks, or, for
+// 0, enough splits that the grid fills about two waves of the SMs, with at least two key
+// blocks per split.  Also returns the key blocks per split.
+int resolve_splits(long long BH, int Nq, int Nk, int d, int requested, int sms, int *blocks_per) {
+    const int BN = d == 64 ? 64 : 128;
+    const int kblocks = (Nk + BN - 1) / BN;
+    int splits;
+    if (requested > 0) {
+        splits = std::min(requested, kblocks);
+    } else {
+        const long long tiles = (long long)((Nq + 127) / 128) * BH;
+        const long long slots = (long long)sms * (d == 64 ? 2 : 1);
+        const long long want = (2 * slots + tiles - 1) / tiles;
+        splits = (int)std::min<long long>(want, std::max(1, kblocks / 2));
+        splits = std::max(1, std::min(splits, 128));
+    }
+    const int bps = (kblocks + splits - 1) / splits;
+    *blocks_per = bps;
+    return (kblocks + bps - 1) / bps;
+}
+
+int current_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return 148;
+    return sms;
+}
+
+size_t splitkv_bytes(long long BH, int Nq, int d, int splits) {
+    if (splits <= 1) return 0;
+    return round256((size_t)splits * BH * Nq * d * 4) + round256((size_t)splits * BH * Nq * 4);
+}
+
+template <int D, bool BF16>
+int launch_splitkv(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                   int Nq, int Nk, float scale, int causal, const int *kv_len, int splits, int bps,
+                   void *workspace, cudaStream_t st, int dev) {
+    if (splits <= 1) {
+        const SplitOut whole;
+        return launch_fwd<D, BF16, false, false>(q, k, v, o, lse, B, H, Nq, Nk, scale, causal,
+                                                 kv_len, nullptr, 0, kNoDropout, whole, st, dev);
+    }
+    const long long bh = (long long)B * H;
+    SplitOut so;
+    so.part_o = static_cast<float *>(workspace);
+    so.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                            round256((size_t)splits * bh * Nq * D * 4));
+    so.num_splits = splits;
+    so.blocks_per_split = bps;
+    int rc = launch_fwd<D, BF16, false, true>(q, k, v, o, lse, B, H, Nq, Nk, scale, causal, kv_len,
+                                              nullptr, 0, kNoDropout, so, st, dev);
+    if (rc != FA_OK) return rc;
+    const long long rows = bh * Nq;
+    cudaError_t e = launch_pdl(fa::fa_splitkv_combine_kernel<D, BF16>,
+                               dim3(grid_for(rows * (D / 4), 256)), dim3(256), 0, st,
+                               (const float *)so.part_o, (const float *)so.part_lse, o, lse, rows,
+                               splits);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "split-KV combine launch");
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -402,19 +484,20 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, floa
     if (rc != FA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
-#define FA_FWD_ARGS q, k, v, o, lse, B, H, N, scale, causal, kv_len, bmask, mask_per_head
+#define FA_FWD_ARGS q, k, v, o, lse, B, H, N, N, scale, causal, kv_len, bmask, mask_per_head
+    const SplitOut whole;
     if (drop) {
         if (d == 64)
-            return bf16 ? launch_fwd<64, true, true>(FA_FWD_ARGS, *drop, st, dev)
-                        : launch_fwd<64, false, true>(FA_FWD_ARGS, *drop, st, dev);
-        return bf16 ? launch_fwd<128, true, true>(FA_FWD_ARGS, *drop, st, dev)
-                    : launch_fwd<128, false, true>(FA_FWD_ARGS, *drop, st, dev);
+            return bf16 ? launch_fwd<64, true, true, false>(FA_FWD_ARGS, *drop, whole, st, dev)
+                        : launch_fwd<64, false, true, false>(FA_FWD_ARGS, *drop, whole, st, dev);
+        return bf16 ? launch_fwd<128, true, true, false>(FA_FWD_ARGS, *drop, whole, st, dev)
+                    : launch_fwd<128, false, true, false>(FA_FWD_ARGS, *drop, whole, st, dev);
     }
     if (d == 64)
-        return bf16 ? launch_fwd<64, true, false>(FA_FWD_ARGS, kNoDropout, st, dev)
-                    : launch_fwd<64, false, false>(FA_FWD_ARGS, kNoDropout, st, dev);
-    return bf16 ? launch_fwd<128, true, false>(FA_FWD_ARGS, kNoDropout, st, dev)
-                : launch_fwd<128, false, false>(FA_FWD_ARGS, kNoDropout, st, dev);
+        return bf16 ? launch_fwd<64, true, false, false>(FA_FWD_ARGS, kNoDropout, whole, st, dev)
+                    : launch_fwd<64, false, false, false>(FA_FWD_ARGS, kNoDropout, whole, st, dev);
+    return bf16 ? launch_fwd<128, true, false, false>(FA_FWD_ARGS, kNoDropout, whole, st, dev)
+                : launch_fwd<128, false, false, false>(FA_FWD_ARGS, kNoDropout, whole, st, dev);
 #undef FA_FWD_ARGS
 }
 
@@ -431,6 +514,50 @@ int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, flo
     if (!block_mask || (mask_per_head != 0 && mask_per_head != 1)) return FA_ERR_INVALID_ARG;
     return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, block_mask,
                       mask_per_head, nullptr, dtype, stream);
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits) {
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || (d != 64 && d != 128) || num_splits < 0 ||
+        num_splits > FA_MAX_SPLITS)
+        return 0;
+    int bps = 0;
+    const long long bh = (long long)B * H;
+    const int splits = resolve_splits(bh, Nq, Nk, d, num_splits, current_sms(), &bps);
+    return splitkv_bytes(bh, Nq, d, splits);
+}
+
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                   int Nq, int Nk, int d, float scale, int causal, const int *kv_len,
+                   int num_splits, int dtype, void *workspace, size_t workspace_bytes,
+                   void *stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > FA_MAX_SPLITS || Nk < 1) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, Nq, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    if ((long long)B * H * (long long)Nk * d > FA_MAX_ELEMENTS) return FA_ERR_UNSUPPORTED;
+    int dev = 0;
+    rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    int bps = 0;
+    const long long bh = (long long)B * H;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+    const int splits = resolve_splits(bh, Nq, Nk, d, num_splits, sms, &bps);
+    const size_t need = splitkv_bytes(bh, Nq, d, splits);
+    if (need > 0 && (!workspace || workspace_bytes < need ||
+                     (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+        return FA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+#define FA_SPLIT_ARGS q, k, v, o, lse, B, H, Nq, Nk, scale, causal, kv_len, splits, bps, workspace, st, dev
+    if (d == 64)
+        return bf16 ? launch_splitkv<64, true>(FA_SPLIT_ARGS) : launch_splitkv<64, false>(FA_SPLIT_ARGS);
+    return bf16 ? launch_splitkv<128, true>(FA_SPLIT_ARGS) : launch_splitkv<128, false>(FA_SPLIT_ARGS);
+#undef FA_SPLIT_ARGS
 }
 
 int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B,

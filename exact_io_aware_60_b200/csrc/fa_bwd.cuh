@@ -235,23 +235,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int kt = blockIdx.x / p.BH;
     const int bh = blockIdx.x - kt * p.BH;
     const int b = bh / p.H;
-    int L = p.N;
-    if (p.kv_len != nullptr) {
-        L = p.kv_len[b];
-        L = L < 0 ? 0 : (L > p.N ? p.N : L);
-    }
-    const int q_begin = p.causal ? kt : 0;
-    // Block-sparse walk: next query tile at or after qi whose (qi, kt) entry is set.
-    const uint8_t *mcol = p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + kt : nullptr;
-    auto next_q = [&](int qi) -> int {
-        if (mcol)
-            while (qi < p.num_tiles && mcol[(size_t)qi * p.num_tiles] == 0) ++qi;
-        return qi;
-    };
-    const int q_first = next_q(q_begin);
-    int n = 0;  // query tiles visited
-    if (kt * 128 < L)
-        for (int qi = q_first; qi < p.num_tiles; qi = next_q(qi + 1)) ++n;
 
     if (warp == C::W_TMA && lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -285,6 +268,25 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     pdl_wait();  // the preprocess kernel's outputs are visible from here on
+
+    // Inputs (key lengths, block mask) are read only after the wait above.
+    int L = p.N;
+    if (p.kv_len != nullptr) {
+        L = p.kv_len[b];
+        L = L < 0 ? 0 : (L > p.N ? p.N : L);
+    }
+    const int q_begin = p.causal ? kt : 0;
+    // Block-sparse walk: next query tile at or after qi whose (qi, kt) entry is set.
+    const uint8_t *mcol = p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + kt : nullptr;
+    auto next_q = [&](int qi) -> int {
+        if (mcol)
+            while (qi < p.num_tiles && mcol[(size_t)qi * p.num_tiles] == 0) ++qi;
+        return qi;
+    };
+    const int q_first = next_q(q_begin);
+    int n = 0;  // query tiles visited
+    if (kt * 128 < L)
+        for (int qi = q_first; qi < p.num_tiles; qi = next_q(qi + 1)) ++n;
 
     if (warp == C::W_TMA) {
         // ------------------------------ TMA producer ------------------------------
@@ -581,16 +583,16 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
                     const float2 d2 = *reinterpret_cast<const float2 *>(dv + cc * 32 + k);
-                    const float2 pp = unpack2<BF16>(Pw[cc * 16 + (k >> 1)]);
                     float dp0 = __uint_as_float(w[k]);
                     float dp1 = __uint_as_float(w[k + 1]);
                     if constexpr (DROP) {
                         if (!((kb[cc] >> (k >> 1)) & 1u)) dp0 = 0.f;
                         if (!((kb[cc] >> ((k >> 1) + 16)) & 1u)) dp1 = 0.f;
                     }
-                    const float ds0 = pp.x * (dp0 - d2.x);
-                    const float ds1 = pp.y * (dp1 - d2.y);
-                    pk[k >> 1] = pack2<BF16>(ds0, ds1);
+                    // dS = P o (dP - D): the difference in fp32, rounded to 16 bits, times
+                    // the 16-bit P pair in one packed multiply
+                    pk[k >> 1] = mul2<BF16>(Pw[cc * 16 + (k >> 1)],
+                                            pack2<BF16>(dp0 - d2.x, dp1 - d2.y));
                 }
                 // dS^T pairs -> TMEM, over dP^T columns this warp has just read; A operand
                 // of dK += dS^T Q.

@@ -54,12 +54,20 @@ namespace fa {
 struct FwdParams {
     float *lse;
     const int *kv_len;
+    // Split-KV partial outputs (SPLIT only): the normalised O and the LSE of each split's
+    // key range, fp32 [num_splits][BH][N][D] and [num_splits][BH][N].
+    float *part_o;
+    float *part_lse;
+    int num_splits;          // 1 without splitting
+    int kv_blocks_per_split; // key blocks per split (0: all)
     // Block-sparse attention: uint8 [heads][T128][T128] (T128 = ceil(N / 128)); a query
     // tile visits only key tiles whose byte is nonzero.  nullptr = dense.
     const uint8_t *bmask;
     long long bmask_bh_stride;  // 0: one mask for every (batch, head)
     int bmask_T;
-    int N;
+    int N;           // query rows
+    int Nk;          // key rows (= N except for the rectangular inference shape)
+    int causal_off;  // Nk - N: query i sees keys j <= i + causal_off under causal masking
     int BH;
     int H;
     int num_q_tiles;
@@ -117,7 +125,9 @@ struct FwdBars {
 
 // DROP: dropout on the probabilities (the mask is regenerated per element from the
 // counter-based generator; the normaliser is the fp32 sum of the undropped values).
-template <int D, bool BF16, bool DROP>
+// SPLIT: the CTA covers one range of key blocks and writes an fp32 partial output (O
+// normalised by that range's own l) and the range's LSE; a combine kernel merges them.
+template <int D, bool BF16, bool DROP, bool SPLIT>
 __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -139,29 +149,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: heaviest causal tiles are launched first.
-    const int tile_rank = blockIdx.x / p.BH;
-    const int bh = blockIdx.x - tile_rank * p.BH;
+    // Work item: (query tile, key split, head); heaviest causal tiles are launched first.
+    const int bh = blockIdx.x % p.BH;
+    const int rest = blockIdx.x / p.BH;
+    const int split = rest % p.num_splits;
+    const int tile_rank = rest / p.num_splits;
     const int qt = p.causal ? (p.num_q_tiles - 1 - tile_rank) : tile_rank;
     const int b = bh / p.H;
-    int L = p.N;
-    if (p.kv_len != nullptr) {
-        L = p.kv_len[b];
-        L = L < 0 ? 0 : (L > p.N ? p.N : L);
-    }
-    int kv_end = L;
-    if (p.causal) kv_end = min(kv_end, (qt + 1) * C::BM);
-    const int T = (kv_end + BN - 1) / BN;  // key blocks in range
-    // Block-sparse walk: next key block at or after j whose tile is set (T if none).
-    const uint8_t *mrow =
-        p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + (size_t)qt * p.bmask_T : nullptr;
-    auto next_block = [&](int j) -> int {
-        if (mrow)
-            while (j < T && mrow[(j * BN) >> 7] == 0) ++j;
-        return j;
-    };
-    const int j_first = next_block(0);
-    const bool any_block = j_first < T;
+    // Softmax warps that hold at least one query row; the others skip the block loop, and
+    // the per-block barriers count only the active ones.
+    const int n_active = min(4, (p.N - qt * C::BM + 31) >> 5);
 
     if (threadIdx.x == 128) {
         tma_prefetch_desc(&tmQ);
@@ -171,9 +168,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bars->q_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[i], 128);
+            mbar_init(&bars->p_full[i], 32 * n_active);
         }
-        mbar_init(&bars->s_read, 128);
+        mbar_init(&bars->s_read, 32 * n_active);
         mbar_init(&bars->o_full, 1);
         for (int i = 0; i < C::NS; ++i) {
             mbar_init(&bars->k_full[i], 1);
@@ -197,6 +194,30 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     pdl_wait();  // inputs written by the previous kernel are visible from here on
+
+    int L = p.Nk;
+    if (p.kv_len != nullptr) {
+        L = p.kv_len[b];
+        L = L < 0 ? 0 : (L > p.Nk ? p.Nk : L);
+    }
+    int kv_end = L;
+    if (p.causal) kv_end = min(kv_end, (qt + 1) * C::BM + p.causal_off);
+    int T = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;  // key blocks in range
+    int j_lo = 0;
+    if (p.kv_blocks_per_split > 0) {  // this split's blocks: [j_lo, T)
+        j_lo = split * p.kv_blocks_per_split;
+        T = min(T, j_lo + p.kv_blocks_per_split);
+    }
+    // Block-sparse walk: next key block at or after j whose tile is set (T if none).
+    const uint8_t *mrow =
+        p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + (size_t)qt * p.bmask_T : nullptr;
+    auto next_block = [&](int j) -> int {
+        if (mrow)
+            while (j < T && mrow[(j * BN) >> 7] == 0) ++j;
+        return j;
+    };
+    const int j_first = next_block(j_lo);
+    const bool any_block = j_first < T;
 
     if (warp == 4) {
         // ------------------------------ TMA producer ------------------------------
@@ -284,7 +305,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float l = 0.f;        // running normaliser
         bool ok = true;
         int jj = 0;  // visited blocks so far
-        for (int j = j_first; j < T; j = next_block(j + 1), ++jj) {
+        const bool active = warp < n_active;
+        for (int j = active ? j_first : T; j < T; j = next_block(j + 1), ++jj) {
             if (!mbar_wait(&bars->s_full[jj % C::SBUF], (jj / C::SBUF) & 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sb = tmem + lane_base + (uint32_t)((jj % C::SBUF) * BN);
@@ -300,24 +322,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tc_fence_before();
                 mbar_arrive(&bars->s_read);
             }
-            const bool need_mask = ((j + 1) * BN > L) || (p.causal && (j + 1) * BN - 1 > qt * C::BM);
+            const bool need_mask =
+                ((j + 1) * BN > L) || (p.causal && (j + 1) * BN - 1 > qt * C::BM + p.causal_off);
             if (need_mask) {
-                const int lim = p.causal ? min(L, row + 1) : L;  // keys < lim are visible
+                // keys < lim are visible
+                const int lim = p.causal ? min(L, row + 1 + p.causal_off) : L;
                 const int c0 = lim - j * BN;
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
                     if (c >= c0) s[c] = -INFINITY;
             }
+            // row max: eight independent chains of three-input maxima, then a short tree
             float mxv[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) mxv[c] = s[c];
+            for (int e = 0; e < 8; ++e) {
+                mxv[e] = fmax3(s[e], s[8 + e], s[16 + e]);
 #pragma unroll
-            for (int c = 8; c < BN; c += 8) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mxv[e] = fmaxf(mxv[e], s[c + e]);
+                for (int c = 24; c + 8 < BN; c += 16) mxv[e] = fmax3(mxv[e], s[c + e], s[c + 8 + e]);
+                if constexpr ((BN / 8 - 3) % 2 == 1) mxv[e] = fmaxf(mxv[e], s[BN - 8 + e]);
             }
-            const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
-                                   fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7]))) * sl2;
+            const float mx = fmax3(fmax3(mxv[0], mxv[1], mxv[2]), fmax3(mxv[3], mxv[4], mxv[5]),
+                                   fmaxf(mxv[6], mxv[7])) * sl2;
             // Lazy rescale: move m only when the max grew by more than 2^8.
             const bool grow = mx > m + 8.0f;
             const bool any_grow = __any_sync(0xffffffffu, grow);
@@ -404,8 +429,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_after();
         }
         const uint32_t ob = tmem + lane_base + C::COL_O;
+        const bool have = active && any_block;  // warp-uniform: TMEM loads are warp-wide
         float l_round = 0.f;
-        if (any_block) {
+        if (have) {
             uint32_t r[16];
             tmem_ld16(ob + D, r);
             l_round = __uint_as_float(r[0]);
@@ -416,12 +442,36 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float inv;
         if constexpr (DROP) inv = (l > 0.f) ? p.drop.keep_scale / l : 0.f;
         else inv = (l > 0.f && l_round > 0.f) ? 1.f / l_round : 0.f;
+        const float lse_row = (l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
+        if constexpr (SPLIT) {
+            // fp32 partial output of this key range, one contiguous row per thread
+            const size_t prow = ((size_t)split * p.BH + bh) * p.N + row;
+            float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * D);
+#pragma unroll
+            for (int c32 = 0; c32 < D / 32; ++c32) {
+                uint32_t r[32];
+                if (have) {
+                    tmem_ld32(ob + c32 * 32, r);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                }
+                if (row < p.N) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[c32 * 8 + i] = make_float4(
+                            __uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                            __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+                }
+            }
+            if (row < p.N) p.part_lse[prow] = lse_row;
+        } else {
 #pragma unroll
         for (int hf = 0; hf < C::HALVES; ++hf) {
             uint32_t w[32];
             {
                 uint32_t r[32];
-                if (any_block) {
+                if (have) {
                     tmem_ld32(ob + hf * 64, r);
                 } else {
 #pragma unroll
@@ -431,7 +481,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int i = 0; i < 16; ++i)
                     w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv,
                                        __uint_as_float(r[2 * i + 1]) * inv);
-                if (any_block) {
+                if (have) {
                     tmem_ld32(ob + hf * 64 + 32, r);
                 }
 #pragma unroll
@@ -455,16 +505,61 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bulk_commit_group();
             bulk_wait_group_read<0>();
         }
-        if (row < p.N) {
-            const float lse = (l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
-            p.lse[(size_t)bh * p.N + row] = lse;
-        }
+        if (row < p.N) p.lse[(size_t)bh * p.N + row] = lse_row;
+        }  // !SPLIT
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// Merges the split-KV partial results: with the per-split LSE_s of a row,
+//   LSE = M + ln sum_s e^(LSE_s - M)  (M = max_s LSE_s),   O = sum_s e^(LSE_s - LSE) O_s,
+// which is the online-softmax (m, l) merge applied once to whole key ranges.  Rows whose
+// every split saw no key get O = 0, LSE = -inf.  D / 4 threads per row, four columns each.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_splitkv_combine_kernel(const float *part_o,
+                                                                const float *part_lse, void *o,
+                                                                float *lse, long long rows,
+                                                                int num_splits) {
+    constexpr int G = D / 4;       // threads per row
+    constexpr int RPW = 32 / G;    // rows per warp step
+    pdl_wait();
+    pdl_launch_dependents();
+    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane % G;
+    for (long long base = (tid >> 5) * RPW; base < rows; base += nwarps * RPW) {
+        const long long r = base + lane / G;
+        if (r >= rows) continue;
+        float mx = -INFINITY;
+        for (int s = 0; s < num_splits; ++s) mx = fmaxf(mx, part_lse[(long long)s * rows + r]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float out_lse = -INFINITY;
+        if (mx != -INFINITY) {
+            float sum = 0.f;
+            for (int s = 0; s < num_splits; ++s) {
+                const float ls = part_lse[(long long)s * rows + r];
+                if (ls == -INFINITY) continue;
+                const float w = __expf(ls - mx);
+                sum += w;
+                const float4 v = reinterpret_cast<const float4 *>(part_o + ((long long)s * rows + r) * D)[g];
+                acc.x = fmaf(w, v.x, acc.x);
+                acc.y = fmaf(w, v.y, acc.y);
+                acc.z = fmaf(w, v.z, acc.z);
+                acc.w = fmaf(w, v.w, acc.w);
+            }
+            const float inv = 1.f / sum;
+            acc = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            out_lse = mx + __logf(sum);
+        }
+        reinterpret_cast<uint2 *>(o)[r * G + g] =
+            make_uint2(pack2<BF16>(acc.x, acc.y), pack2<BF16>(acc.z, acc.w));
+        if (g == 0) lse[r] = out_lse;
+    }
 }
 
 }  // namespace fa

@@ -86,6 +86,11 @@ def lib():
                                          f, u64, u32, i, vp, sz, vp]
             L.fa_dropout_mask.restype = i
             L.fa_dropout_mask.argtypes = [i, i, i, f, u64, u32, vp, vp]
+            L.fa_fwd_splitkv_workspace_bytes.restype = sz
+            L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
+            L.fa_fwd_splitkv.restype = i
+            L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, i, i, vp, sz,
+                                         vp]
             L.fa_bwd_noalloc.restype = i
             L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i,
                                          vp, i, vp]
@@ -295,6 +300,49 @@ def fa_dropout_mask(keep, *, p_drop: float, seed: int, offset: int = 0, stream=N
                                _stream_handle(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_dropout_mask")
+
+
+def fa_fwd_splitkv_workspace_bytes(B: int, H: int, Nq: int, Nk: int, d: int,
+                                   num_splits: int = 0) -> int:
+    return int(lib().fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits))
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, *, scale: float, causal: bool = False, kv_len=None,
+                   num_splits: int = 0, workspace=None, stream=None) -> None:
+    """Inference-shaped forward: q, o [B,H,Nq,d] against k, v [B,H,Nk,d], the key range
+    split over CTAs and merged (see include/fa.h).  ``workspace``: uint8 CUDA tensor of
+    ``fa_fwd_splitkv_workspace_bytes`` bytes (None allowed when that is 0)."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    for name, t, n in (("q", q, Nq), ("k", k, Nk), ("v", v, Nk), ("o", o, Nq)):
+        _check(t, name, (B, H, n, d), q.dtype)
+    _check(lse, "lse", (B, H, Nq), torch.float32)
+    if workspace is not None and (not workspace.is_cuda or workspace.dtype != torch.uint8
+                                  or not workspace.is_contiguous()):
+        raise FAError(FA_ERR_INVALID_ARG, "workspace must be a contiguous uint8 CUDA tensor")
+    rc = lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), B, H, Nq, Nk, d, float(scale), int(bool(causal)),
+                              _kv_ptr(kv_len, B), int(num_splits), _dtype_code(q),
+                              None if workspace is None else workspace.data_ptr(),
+                              0 if workspace is None else workspace.numel(),
+                              _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_splitkv")
+
+
+def forward_splitkv(q, k, v, *, scale: Optional[float] = None, causal: bool = False,
+                    kv_len=None, num_splits: int = 0, stream=None):
+    """Allocates ``o``, ``lse`` and the workspace with torch and runs :func:`fa_fwd_splitkv`."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    B, H, Nq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    n = fa_fwd_splitkv_workspace_bytes(B, H, Nq, k.shape[2], d, num_splits)
+    ws = torch.empty(n, dtype=torch.uint8, device=q.device) if n > 0 else None
+    fa_fwd_splitkv(q, k, v, o, lse, scale=scale, causal=causal, kv_len=kv_len,
+                   num_splits=num_splits, workspace=ws, stream=stream)
+    return o, lse
 
 
 def fa_set_timing_events(which: int, start=None, stop=None) -> None:

@@ -39,13 +39,32 @@ class Workload:
     spike_frac: float = 0.0                # fraction of key positions scaled
     spike_scale: float = 1.0               # factor for those keys (a power of two)
     description: str = ""
+    # Inference shape: Nq queries against N keys (the queries are the last Nq positions of
+    # the sequence); None = training shape with Nq = N.
+    Nq: Optional[int] = None
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
+    @property
+    def n_q(self) -> int:
+        return self.N if self.Nq is None else self.Nq
+
+    @property
+    def inference(self) -> bool:
+        return self.Nq is not None
+
     def nominal_flops(self) -> tuple:
-        """(forward, backward) FLOPs: 4 B H N^2 d forward, 2.5x backward, halved causal."""
+        """(forward, backward) FLOPs: 4 B H N^2 d forward, 2.5x backward, halved causal.
+        Inference shape: 4 d per visible (query, key) pair, i.e. Nq N pairs, less
+        Nq (Nq - 1) / 2 under causal masking (bottom-right aligned)."""
+        if self.inference:
+            pairs = self.n_q * self.N
+            if self.causal:
+                pairs -= self.n_q * (self.n_q - 1) / 2
+            f = 4.0 * self.B * self.H * self.d * pairs
+            return f, 2.5 * f
         f = 4.0 * self.B * self.H * self.N * self.N * self.d
         if self.causal:
             f *= 0.5
@@ -66,6 +85,13 @@ WORKLOADS = {
                           spike_frac=0.01, spike_scale=8.0,
                           description="very long causal: B1 H16 N65536 d128 bf16, 1% of "
                                       "keys x8"),
+    # inference shapes (forward only): new queries against a long key sequence
+    "decode32k": Workload("decode32k", 8, 16, 32768, 128, torch.bfloat16, causal=True, Nq=1,
+                          description="inference decode: B8 H16, 1 query against 32768 keys, "
+                                      "d128 bf16"),
+    "chunk16k": Workload("chunk16k", 1, 16, 16384, 128, torch.bfloat16, causal=True, Nq=512,
+                         description="inference prefill chunk: B1 H16, 512 queries against "
+                                     "16384 keys, d128 bf16 causal"),
 }
 
 
@@ -77,13 +103,15 @@ def custom(name="custom", *, B, H, N, d, dtype=torch.bfloat16, causal=False,
 
 def make_inputs(w: Workload, seed: int = 0, with_grad: bool = True) -> dict:
     """Host (CPU) tensors for workload ``w``: q, k, v, do in ``w.dtype`` (``[B,H,N,d]``,
-    contiguous), ``kv_len`` (int32 ``[B]`` or None), ``spike_keys`` (int64 or None)."""
+    contiguous; q and do ``[B,H,Nq,d]`` for an inference shape), ``kv_len`` (int32 ``[B]``
+    or None), ``spike_keys`` (int64 or None)."""
     g = torch.Generator("cpu").manual_seed(seed)
     shape = (w.B, w.H, w.N, w.d)
-    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    qshape = (w.B, w.H, w.n_q, w.d)
+    q = torch.randn(qshape, generator=g, dtype=torch.float32)
     k = torch.randn(shape, generator=g, dtype=torch.float32)
     v = torch.randn(shape, generator=g, dtype=torch.float32)
-    do = torch.randn(shape, generator=g, dtype=torch.float32) if with_grad else None
+    do = torch.randn(qshape, generator=g, dtype=torch.float32) if with_grad else None
     kv_len = None
     if w.kv_len_range is not None:
         lo, hi = w.kv_len_range

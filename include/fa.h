@@ -158,6 +158,40 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, void *stream);
 
 /*
+ * Inference-shaped forward (aicassindra page, "Inference"; stackzen glossary, where the
+ * savings of the method at inference are cited): Nq queries against Nk keys, Nq usually
+ * much smaller than Nk (decoding, or a chunk of new tokens against a long cache).  The
+ * queries are the last Nq positions of the key sequence:
+ *     key j is visible to query i  iff  j < kv_len[b]  and  (!causal or j <= i + Nk - Nq).
+ * The key range is split into num_splits parts processed by separate CTAs (so that a
+ * short query block still fills the GPU); each part produces its own normalised output
+ * and LSE, and a second kernel merges them with the online-softmax (m, l) rule:
+ *     LSE = M + ln sum_s e^(LSE_s - M),  O = sum_s e^(LSE_s - LSE) O_s,  M = max_s LSE_s.
+ * The result equals fa_fwd's up to floating-point order (with Nq = Nk and num_splits = 1
+ * it is fa_fwd).
+ *   q, o       : DEVICE [B, H, Nq, d] 16-bit; lse: DEVICE [B, H, Nq] fp32.
+ *   k, v       : DEVICE [B, H, Nk, d] 16-bit.
+ *   num_splits : 0 = chosen by the library (about two waves of CTAs, at least two key
+ *                blocks per split), else 1 .. FA_MAX_SPLITS (capped by the number of key
+ *                blocks: 64 keys at d = 64, 128 at d = 128).
+ *   workspace  : DEVICE scratch of fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d,
+ *                num_splits) bytes, 256-byte aligned, owned by the caller (may be NULL when
+ *                that size is 0, i.e. when the call resolves to one split).  The size is
+ *                computed for the current device; call both on the same device.
+ * Returns FA_ERR_INVALID_ARG for the checks of fa_fwd, Nk < 1, num_splits outside
+ * [0, FA_MAX_SPLITS], or a missing / small / misaligned workspace; otherwise as fa_fwd.
+ * Not valid for training: there is no matching backward entry point.
+ */
+#define FA_MAX_SPLITS 256
+
+FA_API size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits);
+
+FA_API int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                          const int *kv_len, int num_splits, int dtype, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
  * Attention with dropout on the probabilities (promptingindex page, "Why attention is
  * memory-bound, not compute-bound": dropout is the op between the softmax and the
  * product with V).  Identical to fa_fwd / fa_bwd except that

@@ -167,3 +167,40 @@ def test_dropout_mask_rejects_bad_arguments_on_host():
     assert L.fa_dropout_mask(1, 1, 0, 0.1, 1, 0, P, None) == fa.FA_ERR_INVALID_ARG
     # more than FA_MAX_ELEMENTS (2^40) mask bytes
     assert L.fa_dropout_mask(1 << 10, 1, 1 << 16, 0.1, 1, 0, P, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_splitkv_workspace_bytes():
+    L = fa.lib()
+    r256 = lambda x: ((x + 255) // 256) * 256
+    # explicit splits: fp32 partial O [splits, B*H, Nq, d] + partial LSE [splits, B*H, Nq]
+    assert L.fa_fwd_splitkv_workspace_bytes(2, 3, 5, 4096, 64, 4) == \
+        r256(4 * 6 * 5 * 64 * 4) + r256(4 * 6 * 5 * 4)
+    # one split needs no workspace; splits are capped by the key blocks (64 keys at d=64)
+    assert L.fa_fwd_splitkv_workspace_bytes(2, 3, 5, 4096, 64, 1) == 0
+    assert L.fa_fwd_splitkv_workspace_bytes(1, 1, 1, 100, 64, 8) == \
+        r256(2 * 1 * 1 * 64 * 4) + r256(2 * 1 * 1 * 4)
+    assert L.fa_fwd_splitkv_workspace_bytes(1, 1, 1, 100, 96, 8) == 0
+    assert L.fa_fwd_splitkv_workspace_bytes(1, 1, 1, 100, 64, 10000) == 0
+
+
+def call_splitkv(**over):
+    a = dict(GOOD, Nq=4, Nk=64, q=P, k=P, v=P, o=P, lse=P, kv=None, splits=0, ws=P,
+             ws_bytes=1 << 30)
+    a.update(over)
+    return fa.lib().fa_fwd_splitkv(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                                   a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"], a["kv"],
+                                   a["splits"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(k=P + 4), fa.FA_ERR_INVALID_ARG),
+    (dict(Nk=0), fa.FA_ERR_INVALID_ARG),
+    (dict(Nq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=257), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+])
+def test_splitkv_rejects_bad_arguments_on_host(over, code):
+    assert call_splitkv(**over) == code

@@ -88,7 +88,7 @@ def test_forward_mask_read_out_exactly(d, N, causal, dtype):
     got = to_f64(gpu["o"]) * L[None, None, :, None] / r
     assert np.all(np.abs(got - counts) < 0.25), np.abs(got - counts).max()
     np.testing.assert_allclose(to_f64(gpu["lse"]), np.broadcast_to(np.log(L), (B, H, N)),
-                               atol=1e-5)
+                               atol=1e-4)
 
 
 @pytest.mark.parametrize("d,N,dtype", [(64, 200, torch.bfloat16), (128, 300, torch.float16)])
