@@ -309,8 +309,14 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         record_cuda_error(e, "cudaFuncSetAttribute(bwd)");
         return FA_ERR_CUDA;
     }
-    const long long grid = (long long)num_tiles * bh;
-    if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    // Persistent: one CTA per SM (or per work item, if fewer) walks the (key tile, head)
+    // items; the kernel takes the grid size into its static schedule.
+    const long long items = (long long)num_tiles * bh;
+    if (items >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+    const long long grid = std::min<long long>(items, sms);
     timing_mark(1, 0, st);
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mdo,
                    mdk, mdv, mdq, p);

@@ -196,7 +196,7 @@ struct BwdBars {
     uint64_t do_full[3];
     uint64_t stage_empty[3];
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
-        dkv_full;
+        dkv_full, dkv_empty;
     uint32_t tmem_base;
 };
 
@@ -231,10 +231,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: key tile kt of head bh; heavier causal tiles (small kt) first.
-    const int kt = blockIdx.x / p.BH;
-    const int bh = blockIdx.x - kt * p.BH;
-    const int b = bh / p.H;
+    // Persistent CTA: work items are (key tile kt, head bh), numbered u = kt * BH + bh so
+    // that heavier causal tiles (small kt) come first.  Round r of CTA c takes item
+    // r * G + c on even rounds and r * G + (G - 1 - c) on odd ones (G = grid size); the
+    // zigzag evens out the causal work.  Every role walks the same list on its own.
 
     if (warp == C::W_TMA && lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -260,6 +260,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 128);
         mbar_init(&bars->dkv_full, 1);
+        mbar_init(&bars->dkv_empty, 256);
         fence_mbar_init();
     }
     if (warp == C::W_MMA) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
@@ -270,35 +271,45 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     pdl_wait();  // the preprocess kernel's outputs are visible from here on
 
     // Inputs (key lengths, block mask) are read only after the wait above.
-    int L = p.N;
-    if (p.kv_len != nullptr) {
-        L = p.kv_len[b];
-        L = L < 0 ? 0 : (L > p.N ? p.N : L);
-    }
-    const int q_begin = p.causal ? kt : 0;
+    struct Item {
+        int kt, bh, L;        // key tile, head, valid keys of the sequence
+        int q_first, n;       // first visited query tile, number of visited query tiles
+        const uint8_t *mcol;  // block-mask column of kt (nullptr: dense)
+    };
     // Block-sparse walk: next query tile at or after qi whose (qi, kt) entry is set.
-    const uint8_t *mcol = p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + kt : nullptr;
-    auto next_q = [&](int qi) -> int {
-        if (mcol)
-            while (qi < p.num_tiles && mcol[(size_t)qi * p.num_tiles] == 0) ++qi;
+    auto next_q = [&](const Item &it, int qi) -> int {
+        if (it.mcol)
+            while (qi < p.num_tiles && it.mcol[(size_t)qi * p.num_tiles] == 0) ++qi;
         return qi;
     };
-    const int q_first = next_q(q_begin);
-    int n = 0;  // query tiles visited
-    if (kt * 128 < L)
-        for (int qi = q_first; qi < p.num_tiles; qi = next_q(qi + 1)) ++n;
+    auto item_at = [&](int r, Item &it) -> bool {
+        const int G = (int)gridDim.x;
+        const int u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        if (u >= p.num_tiles * p.BH) return false;
+        it.kt = u / p.BH;
+        it.bh = u - it.kt * p.BH;
+        int L = p.N;
+        if (p.kv_len != nullptr) {
+            L = p.kv_len[it.bh / p.H];
+            L = L < 0 ? 0 : (L > p.N ? p.N : L);
+        }
+        it.L = L;
+        it.mcol = p.bmask ? p.bmask + (size_t)it.bh * p.bmask_bh_stride + it.kt : nullptr;
+        it.q_first = next_q(it, p.causal ? it.kt : 0);
+        it.n = 0;
+        if (it.kt * 128 < L)
+            for (int qi = it.q_first; qi < p.num_tiles; qi = next_q(it, qi + 1)) ++it.n;
+        return true;
+    };
 
     if (warp == C::W_TMA) {
         // ------------------------------ TMA producer ------------------------------
-        if (lane == 0 && n > 0) {
-            mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
-            for (int hf = 0; hf < C::HALVES; ++hf) {
-                tma_load_3d(sK + hf * C::HALF, &tmK, &bars->kv_full, hf * 64, kt * 128, bh);
-                tma_load_3d(sV + hf * C::HALF, &tmV, &bars->kv_full, hf * 64, kt * 128, bh);
-            }
-            for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
-                const int s = i % C::QS;
-                if (i >= C::QS && !mbar_wait(&bars->stage_empty[s], ((i / C::QS) - 1) & 1)) break;
+        if (lane == 0) {
+            // Q_i, dO_i (+ LSE_i, D_i) of global iteration g into ring stage g % QS.
+            auto load_q = [&](int g, int qi, int bh) -> bool {
+                const int s = g % C::QS;
+                if (g >= C::QS && !mbar_wait(&bars->stage_empty[s], ((g / C::QS) - 1) & 1))
+                    return false;
                 const size_t vec_off = (size_t)bh * p.Npad + (size_t)qi * 128;
                 mbar_arrive_expect_tx(&bars->q_full[s], C::TILE + 512);
                 for (int hf = 0; hf < C::HALVES; ++hf)
@@ -310,11 +321,34 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tma_load_3d(sdO + s * C::TILE + hf * C::HALF, &tmdO, &bars->do_full[s],
                                 hf * 64, qi * 128, bh);
                 bulk_load(sDv + s * 128, p.dvec + vec_off, 512, &bars->do_full[s]);
+                return true;
+            };
+            bool ok = true;
+            int gi = 0, tn = 0;  // global iteration, items with work so far
+            Item it;
+            for (int r = 0; ok && item_at(r, it); ++r) {
+                if (it.n == 0) continue;
+                // The first Q/dO tiles of this item go in as soon as their stages free up
+                // (while the previous item still runs); K and V wait for the previous
+                // item's last MMA.
+                const int pre = min(it.n, C::QS - 1);
+                int qi = it.q_first;
+                for (int i = 0; ok && i < pre; ++i, qi = next_q(it, qi + 1)) ok = load_q(gi + i, qi, it.bh);
+                if (ok && tn > 0) ok = mbar_wait(&bars->dkv_full, (tn - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
+                for (int hf = 0; hf < C::HALVES; ++hf) {
+                    tma_load_3d(sK + hf * C::HALF, &tmK, &bars->kv_full, hf * 64, it.kt * 128, it.bh);
+                    tma_load_3d(sV + hf * C::HALF, &tmV, &bars->kv_full, hf * 64, it.kt * 128, it.bh);
+                }
+                for (int i = pre; ok && i < it.n; ++i, qi = next_q(it, qi + 1)) ok = load_q(gi + i, qi, it.bh);
+                gi += it.n;
+                ++tn;
             }
         }
     } else if (warp == C::W_MMA) {
         // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0 && n > 0) {
+        if (lane == 0) {
             constexpr uint32_t kIdescSq = idesc_f16(BF16, false, false, 128, 128);  // S^T, dP^T
             constexpr uint32_t kIdescTs = idesc_f16(BF16, false, true, 128, D);     // dV, dK
             constexpr uint32_t kIdescDq = idesc_f16(BF16, true, true, 128, D);      // dQ
@@ -347,71 +381,88 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                            (acc || kk > 0) ? 1u : 0u);
             };
             auto stage_off = [](int st) { return (uint64_t)((st * C::TILE) >> 4); };
-            bool ok = mbar_wait(&bars->kv_full, 0);
-            ok = ok && mbar_wait(&bars->q_full[0], 0);
-            tc_fence_after();
-            if (ok) {
-                mma_square(tmem + C::COL_S, k_kmaj, q_kmaj);
-                mma_commit(&bars->s_full);
-                ok = mbar_wait(&bars->do_full[0], 0);
+            bool ok = true;
+            int gi = 0, tn = 0;  // global iteration, items with work so far
+            Item it;
+            for (int r = 0; ok && item_at(r, it); ++r) {
+                const int n = it.n;
+                if (n == 0) continue;
+                if (!mbar_wait(&bars->kv_full, tn & 1)) break;
                 tc_fence_after();
-            }
-            if (ok) {
-                mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj);
-                mma_commit(&bars->dp_full);
-            }
-            for (int i = 0; ok && i < n; ++i) {
-                const int s = i % C::QS;
-                if (C::P_OWN && i + 1 < n) {
-                    // S_{i+1} overwrites S_i as soon as every P/dS warp has read it.
-                    const int s1 = (i + 1) % C::QS;
-                    if (!mbar_wait(&bars->s_free, i & 1)) break;
-                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) / C::QS) & 1)) break;
+                // First S^T and dP^T of the item.  S^T overwrites the previous item's last
+                // S^T once the P/dS warps have read it (d = 64); at d = 128 it overwrites the
+                // previous P^T, which the (earlier issued) dV MMA has consumed.  dP^T at
+                // d = 128 shares its columns with dQ: the previous dQ must be drained.
+                {
+                    const int s0 = gi % C::QS;
+                    if (C::P_OWN && gi > 0 && !mbar_wait(&bars->s_free, (gi - 1) & 1)) break;
+                    if (!mbar_wait(&bars->q_full[s0], (gi / C::QS) & 1)) break;
                     tc_fence_after();
-                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
+                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s0));
                     mma_commit(&bars->s_full);
-                }
-                if (!mbar_wait(&bars->p_full, i & 1)) break;
-                tc_fence_after();
-                mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE, do_mn + stage_off(s),
-                           i > 0);
-                mma_commit(&bars->p_free);
-                if (!C::P_OWN && i + 1 < n) {
-                    // P^T_i lives in the S^T columns: S_{i+1} follows dV_i.
-                    const int s1 = (i + 1) % C::QS;
-                    if (!mbar_wait(&bars->q_full[s1], ((i + 1) / C::QS) & 1)) break;
+                    if (D == 128 && gi > 0 && !mbar_wait(&bars->dq_empty, (gi - 1) & 1)) break;
+                    if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
                     tc_fence_after();
-                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
-                    mma_commit(&bars->s_full);
-                }
-                if (!mbar_wait(&bars->ds_full, i & 1)) break;
-                tc_fence_after();
-                mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
-                           q_mn + stage_off(s), i > 0);
-                if (D == 64 && i > 0) {
-                    if (!mbar_wait(&bars->dq_empty, (i - 1) & 1)) break;
-                    tc_fence_after();
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
-                           k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
-                mma_commit(&bars->dq_full);
-                mma_commit(&bars->ds_empty);
-                mma_commit(&bars->stage_empty[s]);
-                if (i + 1 < n) {
-                    const int s1 = (i + 1) % C::QS;
-                    if (D == 128) {
-                        // dQ_i lives in the dP^T columns: wait until it has been drained.
-                        if (!mbar_wait(&bars->dq_empty, i & 1)) break;
-                    }
-                    if (!mbar_wait(&bars->do_full[s1], ((i + 1) / C::QS) & 1)) break;
-                    tc_fence_after();
-                    mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
+                    mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s0));
                     mma_commit(&bars->dp_full);
                 }
+                for (int i = 0; i < n; ++i) {
+                    const int g = gi + i;  // global iteration: ring stage and barrier phases
+                    const int s = g % C::QS;
+                    const int s1 = (g + 1) % C::QS;
+                    if (C::P_OWN && i + 1 < n) {
+                        // S_{i+1} overwrites S_i as soon as every P/dS warp has read it.
+                        if (!mbar_wait(&bars->s_free, g & 1) ||
+                            !mbar_wait(&bars->q_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
+                        mma_commit(&bars->s_full);
+                    }
+                    if (!mbar_wait(&bars->p_full, g & 1)) { ok = false; break; }
+                    // dV and dK start from zero in this item: the previous item's epilogue
+                    // must have read them out of TMEM.
+                    if (i == 0 && tn > 0 && !mbar_wait(&bars->dkv_empty, (tn - 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE,
+                               do_mn + stage_off(s), i > 0);
+                    mma_commit(&bars->p_free);
+                    if (!C::P_OWN && i + 1 < n) {
+                        // P^T_i lives in the S^T columns: S_{i+1} follows dV_i.
+                        if (!mbar_wait(&bars->q_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
+                        mma_commit(&bars->s_full);
+                    }
+                    if (!mbar_wait(&bars->ds_full, g & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
+                               q_mn + stage_off(s), i > 0);
+                    if (D == 64 && g > 0) {
+                        if (!mbar_wait(&bars->dq_empty, (g - 1) & 1)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
+                               k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
+                    mma_commit(&bars->dq_full);
+                    mma_commit(&bars->ds_empty);
+                    mma_commit(&bars->stage_empty[s]);
+                    if (i + 1 < n) {
+                        if (D == 128) {
+                            // dQ_i lives in the dP^T columns: wait until it has been drained.
+                            if (!mbar_wait(&bars->dq_empty, g & 1)) { ok = false; break; }
+                        }
+                        if (!mbar_wait(&bars->do_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
+                        mma_commit(&bars->dp_full);
+                    }
+                }
+                mma_commit(&bars->dkv_full);
+                gi += n;
+                ++tn;
             }
-            mma_commit(&bars->dkv_full);
         }
     } else if (warp >= C::W_DQ0) {
         // ------------------------------ dQ drain ----------------------------------
@@ -419,8 +470,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int r = quarter * 32 + lane;          // query row in the tile = TMEM lane
         const int gt = threadIdx.x - C::W_DQ0 * 32;  // 0..127 inside this warpgroup
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
-            if (!mbar_wait(&bars->dq_full, i & 1)) break;
+        bool ok = true;
+        int gi = 0;
+        Item it;
+        for (int rr = 0; ok && item_at(rr, it); ++rr) {
+        const int bh = it.bh;
+        for (int i = 0, qi = it.q_first; i < it.n; ++i, qi = next_q(it, qi + 1)) {
+            if (!mbar_wait(&bars->dq_full, (gi + i) & 1)) { ok = false; break; }
             tc_fence_after();
             if constexpr (C::DQ_TMA) {
                 if (gt == 0) bulk_wait_group_read<0>();
@@ -465,6 +521,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mbar_arrive(&bars->dq_empty);
             }
         }
+        gi += it.n;
+        }
         if constexpr (C::DQ_TMA) {
             if (gt == 0) bulk_wait_group<0>();
         }
@@ -473,13 +531,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int quarter = warp & 3;
         const int h = warp >> 2;             // query half: columns 64h .. 64h + 63
         const int t = quarter * 32 + lane;   // key row in the tile = TMEM lane
-        const int key = kt * 128 + t;
-        const bool key_ok = key < L;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
-        for (int i = 0, qi = q_first; i < n; ++i, qi = next_q(qi + 1)) {
-            const int s = i % C::QS;
+        int gi = 0, tn = 0;  // global iteration, items with work so far
+        Item it;
+        for (int rr = 0; item_at(rr, it); ++rr) {
+        const int kt = it.kt, bh = it.bh, L = it.L, n = it.n;
+        const bool key_ok = kt * 128 + t < L;
+        for (int i = 0, qi = it.q_first; ok && i < n; ++i, qi = next_q(it, qi + 1)) {
+            const int g = gi + i;  // global iteration: ring stage and barrier phases
+            const int s = g % C::QS;
             // Dropout keep bits of this key row against queries 64h .. 64h + 63 of tile qi:
             // bit m of kb[u] = query 32u + 2m, bit m + 16 = query 32u + 2m + 1.  Each lane
             // of a half-warp draws the Philox blocks of two queries for the half-warp's
@@ -499,7 +561,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     kb[u] = transpose16x16_halfwarp(a | (c << 16), lane);
                 }
             }
-            if (!mbar_wait(&bars->s_full, i & 1) || !mbar_wait(&bars->q_full[s], (i / C::QS) & 1)) {
+            if (!mbar_wait(&bars->s_full, g & 1) || !mbar_wait(&bars->q_full[s], (g / C::QS) & 1)) {
                 ok = false;
                 break;
             }
@@ -548,7 +610,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                 }
             }
-            if (C::P_OWN && i > 0 && !mbar_wait(&bars->p_free, (i - 1) & 1)) {  // dV_{i-1} read P
+            if (C::P_OWN && g > 0 && !mbar_wait(&bars->p_free, (g - 1) & 1)) {  // dV_{g-1} read P
                 ok = false;
                 break;
             }
@@ -567,8 +629,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(&bars->p_full);
 
-            if (!mbar_wait(&bars->dp_full, i & 1) || !mbar_wait(&bars->do_full[s], (i / C::QS) & 1) ||
-                (i > 0 && !mbar_wait(&bars->ds_empty, (i - 1) & 1))) {
+            if (!mbar_wait(&bars->dp_full, g & 1) || !mbar_wait(&bars->do_full[s], (g / C::QS) & 1) ||
+                (g > 0 && !mbar_wait(&bars->ds_empty, (g - 1) & 1))) {
                 ok = false;
                 break;
             }
@@ -612,58 +674,78 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_arrive(&bars->ds_full);
         }
 
-        // ------------------------------ epilogue: dK, dV ------------------------------
-        pdl_launch_dependents();
+        // ------------------------------ epilogue of the item: dK, dV ---------------------
+        // All 256 threads agree on whether to go on (a bounded wait may have failed).
+        ok = named_bar_and(1, 256, ok);
+        Item nxt;
+        if (!item_at(rr + 1, nxt)) pdl_launch_dependents();  // this CTA's last item
         if (ok && n > 0) {
-            ok = mbar_wait(&bars->dkv_full, 0);
+            ok = mbar_wait(&bars->dkv_full, tn & 1);
             tc_fence_after();
         }
-        // Staging: the first Q / dO stage buffers are free once every MMA is done.  Each
-        // warp converts its lane quarter's D/2 columns of dV and dK.
-        uint8_t *stage_v = sQ;
-        uint8_t *stage_k = sdO;
+        // Staging in the dS buffer (free: every MMA of the item is done; 32 KB): both
+        // 16-bit tiles at d = 64, one tile per round at d = 128.  Each warp converts its
+        // lane quarter's D/2 columns.
         constexpr int HCOLS = D / 2;  // columns of this warp's half
+        constexpr int ROUNDS = (D == 64) ? 1 : 2;
 #pragma unroll
-        for (int which = 0; which < 2; ++which) {
-            const uint32_t col = (which == 0 ? C::COL_DV : C::COL_DK) + h * HCOLS;
-            float mul = which == 0 ? 1.f : p.scale;
-            if constexpr (DROP) mul = which == 0 ? p.dv_mul : p.dk_mul;
-            uint8_t *stage = which == 0 ? stage_v : stage_k;
+        for (int round = 0; round < ROUNDS; ++round) {
 #pragma unroll
-            for (int c32 = 0; c32 < HCOLS / 32; ++c32) {
-                uint32_t w[32];
-                if (n > 0) {
-                    tmem_ld32(tmem + lane_base + col + c32 * 32, w);
-                } else {
+            for (int which = 0; which < 2; ++which) {
+                if (ROUNDS == 2 && which != round) continue;
+                const uint32_t col = (which == 0 ? C::COL_DV : C::COL_DK) + h * HCOLS;
+                float mul = which == 0 ? 1.f : p.scale;
+                if constexpr (DROP) mul = which == 0 ? p.dv_mul : p.dk_mul;
+                uint8_t *stage = sdS + (ROUNDS == 1 ? which * C::HALF : 0);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) w[k] = 0u;
+                for (int c32 = 0; c32 < HCOLS / 32; ++c32) {
+                    uint32_t w[32];
+                    if (n > 0) {
+                        tmem_ld32(tmem + lane_base + col + c32 * 32, w);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) w[k] = 0u;
+                    }
+                    uint32_t wv[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        wv[k] = pack2<BF16>(__uint_as_float(w[2 * k]) * mul,
+                                            __uint_as_float(w[2 * k + 1]) * mul);
+                    // element e = h * HCOLS + c32 * 32 .. + 31 of row t: 128-byte block e / 64,
+                    // 16-byte chunks (e % 64) / 8 .. + 3
+                    const int e0 = h * HCOLS + c32 * 32;
+                    uint8_t *rowp = stage + (e0 >> 6) * C::HALF + t * 128;
+                    const int ch0 = (e0 & 63) >> 3;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4 *>(rowp + (((ch0 + c) ^ (t & 7)) << 4)) =
+                            make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
                 }
-                uint32_t wv[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    wv[k] = pack2<BF16>(__uint_as_float(w[2 * k]) * mul,
-                                        __uint_as_float(w[2 * k + 1]) * mul);
-                // element e = h * HCOLS + c32 * 32 .. + 31 of row t: 128-byte block e / 64,
-                // 16-byte chunks (e % 64) / 8 .. + 3
-                const int e0 = h * HCOLS + c32 * 32;
-                uint8_t *rowp = stage + (e0 >> 6) * C::HALF + t * 128;
-                const int ch0 = (e0 & 63) >> 3;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4 *>(rowp + (((ch0 + c) ^ (t & 7)) << 4)) =
-                        make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
             }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 256);
-        if (threadIdx.x == 0) {
-            for (int hf = 0; hf < C::HALVES; ++hf) {
-                tma_store_3d(&tmdV, stage_v + hf * C::HALF, hf * 64, kt * 128, bh);
-                tma_store_3d(&tmdK, stage_k + hf * C::HALF, hf * 64, kt * 128, bh);
+            if (round == ROUNDS - 1 && n > 0) {
+                // dK, dV are out of TMEM: the next item's first dV / dK MMA may start
+                tc_fence_before();
+                mbar_arrive(&bars->dkv_empty);
             }
-            bulk_commit_group();
-            bulk_wait_group_read<0>();
+            fence_proxy_async_smem();
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 0) {
+                for (int which = 0; which < 2; ++which) {
+                    if (ROUNDS == 2 && which != round) continue;
+                    const uint8_t *stage = sdS + (ROUNDS == 1 ? which * C::HALF : 0);
+                    for (int hf = 0; hf < C::HALVES; ++hf)
+                        tma_store_3d(which == 0 ? &tmdV : &tmdK, stage + hf * C::HALF, hf * 64,
+                                     kt * 128, bh);
+                }
+                bulk_commit_group();
+                bulk_wait_group_read<0>();  // the dS buffer is reused right after
+            }
+            named_bar_sync(1, 256);
         }
+        gi += n;
+        if (n > 0) ++tn;
+        if (!ok) break;
+        }  // items
     }
 
     tc_fence_before();
