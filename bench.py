@@ -63,11 +63,19 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def step_flops(w, block_mask=None) -> tuple:
+def quantise_e4m3(x):
+    """Per-tensor E4M3 quantisation of a host tensor: (bytes, scale factor)."""
+    import torch
+    s = float(x.float().abs().max()) / 448.0
+    return (x.float() / s).to(torch.float8_e4m3fn), s
+
+
+def step_flops(w, block_mask=None, fwd_only=False) -> tuple:
     """(forward, backward, total) FLOPs of one step.  Dense: the nominal count.  With a
     block mask: 4 d per visible (query, key) pair forward and 10 d backward (the work the
-    kernels actually do; masked blocks are skipped).  Inference shape: forward only."""
-    if w.inference:
+    kernels actually do; masked blocks are skipped).  Inference shape or FP8: forward
+    only."""
+    if w.inference or fwd_only:
         f = w.nominal_flops()[0]
         return f, 0.0, f
     if block_mask is None:
@@ -232,9 +240,20 @@ def inference_bytes(w) -> float:
     return float(w.B * w.H * (2 * w.N * w.d * e + 2 * w.n_q * w.d * e + 4 * w.n_q))
 
 
-def alloc_set(w, inp, dev):
+def alloc_set(w, inp, dev, fp8=False):
     import torch
     from exact_io_aware_60_b200 import fa
+    if fp8:
+        s = {}
+        for n in ("q", "k", "v"):
+            x8, sc = quantise_e4m3(inp[n])
+            s[n] = x8.to(dev)
+            s[n + "_scale"] = sc
+        s["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
+        s["o"] = torch.empty(s["q"].shape, dtype=torch.bfloat16, device=dev)
+        s["lse"] = torch.empty(s["q"].shape[:-1], dtype=torch.float32, device=dev)
+        s["fp8"] = True
+        return s
     if w.inference:
         s = {n: inp[n].to(dev) for n in ("q", "k", "v")}
         s["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
@@ -253,11 +272,17 @@ def alloc_set(w, inp, dev):
 
 
 def set_bytes(s) -> int:
-    return sum(t.numel() * t.element_size() for n, t in s.items() if t is not None)
+    import torch
+    return sum(t.numel() * t.element_size() for n, t in s.items() if isinstance(t, torch.Tensor))
 
 
 def run_step(w, s, stream=None):
     from exact_io_aware_60_b200 import fa
+    if s.get("fp8"):
+        fa.fa_fwd_fp8(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale,
+                      q_scale=s["q_scale"], k_scale=s["k_scale"], v_scale=s["v_scale"],
+                      causal=w.causal, kv_len=s["kv_len"], stream=stream)
+        return
     if w.inference:
         fa.fa_fwd_splitkv(s["q"], s["k"], s["v"], s["o"], s["lse"], scale=w.scale,
                           causal=w.causal, kv_len=s["kv_len"], num_splits=0,
@@ -285,12 +310,17 @@ def run_step(w, s, stream=None):
               stream=stream)
 
 
-def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0) -> dict:
+def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0, fp8_set=None) -> dict:
     """The oracle (as it stands) on whole heads of the workload until ``budget_s`` of CPU
     time has passed (at least one head)."""
     import oracle
-    q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
-    do = None if w.inference else inp["do"].double().numpy()
+    if fp8_set is not None:  # the values the E4M3 inputs represent
+        q, k, v = (fp8_set[n].cpu().double().numpy() * fp8_set[n + "_scale"]
+                   for n in ("q", "k", "v"))
+        do = None
+    else:
+        q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+        do = None if w.inference else inp["do"].double().numpy()
     kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     t0 = time.perf_counter()
@@ -305,10 +335,10 @@ def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0) -> dict
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    flops = step_flops(w)[2] * done / (w.B * w.H)
+    flops = step_flops(w, fwd_only=do is None)[2] * done / (w.B * w.H)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": f"fp64 oracle {'forward' if w.inference else 'forward+backward'} of "
+            "sample": f"fp64 oracle {'forward' if do is None else 'forward+backward'} of "
                       f"{done} of {w.B * w.H} (batch, head) "
                       f"pairs of the {w.name} workload"
                       + (f" with dropout p={dropout_p}" if dropout_p else "")
@@ -328,14 +358,15 @@ def bench_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = W.WORKLOADS[args.workload]
     mask_np = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
-    f_fwd, f_bwd, f_step = step_flops(w, mask_np)
+    f_fwd, f_bwd, f_step = step_flops(w, mask_np, fwd_only=args.fp8)
 
-    inp = W.make_inputs(w, seed=rank_seed(rank))
-    first = alloc_set(w, inp, dev)
+    inp = W.make_inputs(w, seed=rank_seed(rank), with_grad=not args.fp8)
+    first = alloc_set(w, inp, dev, fp8=args.fp8)
     per_set = set_bytes(first)
     l2 = 126 * 2 ** 20
     nsets = max(2, math.ceil(2 * l2 / per_set) + 1)
-    sets = [first] + [alloc_set(w, W.make_inputs(w, seed=rank_seed(rank) + i), dev)
+    sets = [first] + [alloc_set(w, W.make_inputs(w, seed=rank_seed(rank) + i,
+                                                 with_grad=not args.fp8), dev, fp8=args.fp8)
                       for i in range(1, nsets)]
     if mask_np is not None:
         mask_t = torch.from_numpy(mask_np).to(dev)
@@ -403,15 +434,19 @@ def bench_ours(args, rank, world, local_rank):
     ms = start.elapsed_time(end)
     max_ms = max_over_ranks(ms, dev if world > 1 else None)
     k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / len(evs[0])
-    k_bwd = 0.0 if w.inference else sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
+    fwd_only = w.inference or args.fp8
+    k_bwd = 0.0 if fwd_only else sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
     value = whole_job_tflops(f_step, world, K, max_ms)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        in_names = ("q", "k", "v") if w.inference else ("q", "k", "v", "do")
-        out_names = ("o", "lse") if w.inference else ("o", "lse", "dq", "dk", "dv")
-        host = {n: inp[n].pin_memory() for n in in_names}
+        in_names = ("q", "k", "v") if fwd_only else ("q", "k", "v", "do")
+        out_names = ("o", "lse") if fwd_only else ("o", "lse", "dq", "dk", "dv")
+        if args.fp8:
+            host = {n: first[n].cpu().pin_memory() for n in in_names}
+        else:
+            host = {n: inp[n].pin_memory() for n in in_names}
         outs = {n: torch.empty(first[n].shape, dtype=first[n].dtype, pin_memory=True)
                 for n in out_names}
         Ke = max(3, min(K, args.e2e_steps))
@@ -445,6 +480,8 @@ def bench_ours(args, rank, world, local_rank):
     sustained = ms > 1000.0
     peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
     peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    if args.fp8:
+        peak *= 2.0  # E4M3 dense peak: the measured bf16 figure x the nominal ratio 4.5 / 2.25
     # the dominant kernel is the one with the larger device time per step
     if k_bwd >= k_fwd:
         dom_name, dom_flops, dom_ms = "fa_bwd_kernel", f_bwd, k_bwd
@@ -453,7 +490,8 @@ def bench_ours(args, rank, world, local_rank):
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peak_src} {peak_key}",
+                "peak_source": f"{peak_src} {peak_key}"
+                               + (" x 2 (e4m3 / bf16 nominal)" if args.fp8 else ""),
                 "flops_per_launch": dom_flops, "launch_ms": dom_ms,
                 "launches_timed": len(evs[0]),
                 "traffic": profile_traffic(dom_name, w.name)}
@@ -467,17 +505,19 @@ def bench_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_sample(w, inp, args.cpu_seconds, args.dropout)
+        cpu = cpu_baseline_sample(w, inp, args.cpu_seconds, args.dropout,
+                                  fp8_set=first if args.fp8 else None)
 
     per_rank_value = f_step * K / (ms * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16"}[w.dtype],
+        "dtype": "e4m3" if args.fp8 else {torch.bfloat16: "bf16", torch.float16: "f16"}[w.dtype],
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
         "config": {"workload": w.description
-                   + (", inference forward (split-KV)" if w.inference else ", forward + backward")
+                   + (", E4M3 inputs (per-tensor scales), forward only" if args.fp8 else
+                      ", inference forward (split-KV)" if w.inference else ", forward + backward")
                    + (", block-sparse local+global pattern" if args.block_sparse else "")
                    + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
                    "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
@@ -487,12 +527,13 @@ def bench_ours(args, rank, world, local_rank):
                          "rotated so each step reads data evicted from the 126 MB L2"},
         "pct_of_peak": 100.0 * per_rank_value / peak,
         "kernels": ({"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12}}
-                    if w.inference else
+                    if fwd_only else
                     {"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12},
                      "fa_bwd_kernel": {"ms": k_bwd, "tflops": f_bwd / (k_bwd * 1e-3) / 1e12}}),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": ((1 + int(first.get("ws_split") is not None)) * K if w.inference
+        "gpu_launches": (K if args.fp8 else
+                         (1 + int(first.get("ws_split") is not None)) * K if w.inference
                          else 4 * K),
         "clocks": clk,
         "cpu_baseline": cpu,
@@ -513,14 +554,21 @@ def bench_reference(args):
     import oracle
     from exact_io_aware_60_b200 import workloads as W
     w = W.WORKLOADS[args.workload]
-    inp = W.make_inputs(w, seed=0)
-    q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
-    do = None if w.inference else inp["do"].double().numpy()
+    inp = W.make_inputs(w, seed=0, with_grad=not args.fp8)
+    if args.fp8:  # the values the E4M3 inputs represent
+        q, k, v = (x8.double().numpy() * sc for x8, sc in
+                   (quantise_e4m3(inp[n]) for n in ("q", "k", "v")))
+        do = None
+    else:
+        q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+        do = None if w.inference else inp["do"].double().numpy()
     kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     total = args.steps + args.warmup
     nq = w.n_q
     rows_per_step = nq if total <= 300 else max(min(16, nq), (nq * 300) // total)
+    # about 2^22 score rows x keys per step at most, so a step stays a fraction of a second
+    rows_per_step = min(rows_per_step, max(16, (1 << 22) // w.N))
     rng = np.random.default_rng(0)
     off = w.N - nq  # inference shape: queries are the last nq positions
 
@@ -536,7 +584,7 @@ def bench_reference(args):
                 for kt in np.nonzero(bmask[i // 128])[0]:
                     vis += max(0, min(lim, (kt + 1) * 128) - kt * 128)
         # 4d forward (+ 10d backward) per visible score
-        return (4.0 if w.inference else 14.0) * w.d * vis
+        return (4.0 if do is None else 14.0) * w.d * vis
 
     def one(i):
         b, h = heads[i % len(heads)]
@@ -557,7 +605,7 @@ def bench_reference(args):
         fl += one(args.warmup + i)
     dt = time.perf_counter() - t0
     value = fl / dt / 1e12
-    sample = (f"fp64 oracle {'forward' if w.inference else 'forward+backward'} of "
+    sample = (f"fp64 oracle {'forward' if do is None else 'forward+backward'} of "
               f"{rows_per_step} query rows of one (batch, head) pair per step, {w.name} workload")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
@@ -565,7 +613,8 @@ def bench_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
         "config": {"workload": w.description
-                   + (", inference forward (split-KV)" if w.inference else ", forward + backward")
+                   + (", E4M3 inputs (per-tensor scales), forward only" if args.fp8 else
+                      ", inference forward (split-KV)" if w.inference else ", forward + backward")
                    + (", block-sparse local+global pattern" if args.block_sparse else "")
                    + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
                    "B": w.B, "H": w.H,
@@ -594,7 +643,11 @@ def main(argv=None):
                          "(FLOPs counted over the visible pairs only)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="measure the dropout path with this drop probability")
+    ap.add_argument("--fp8", action="store_true",
+                    help="measure the E4M3 forward (d = 128 workloads; forward only)")
     args = ap.parse_args(argv)
+    if args.fp8 and (args.dropout or args.block_sparse):
+        ap.error("--fp8 measures the plain E4M3 forward")
     if args.dropout and args.block_sparse:
         ap.error("--dropout and --block-sparse measure different paths; pick one")
     if not (0.0 <= args.dropout < 255.5 / 256):

@@ -153,20 +153,23 @@ struct SplitOut {
     int blocks_per_split = 0;
 };
 
-template <int D, bool BF16, bool DROP, bool SPLIT>
+template <int D, bool BF16, bool DROP, bool SPLIT, bool F8 = false>
 int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
                int N, int Nk, float scale, int causal, const int *kv_len, const uint8_t *bmask,
                int mask_per_head, const fa::DropoutParams &drop, const SplitOut &so,
-               cudaStream_t st, int dev) {
-    using C = fa::FwdCfg<D>;
+               cudaStream_t st, int dev, float out_scale = 1.f) {
+    using C = std::conditional_t<F8, fa::FwdCfgF8, fa::FwdCfg<D>>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    // inputs: 16-bit with 64-element (128-byte) boxes, or E4M3 bytes with 128-element boxes
+    const CUtensorMapDataType dti = F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : dt;
+    const int ie = F8 ? 1 : 2, ib = F8 ? 128 : 64;
     const long long bh = (long long)B * H;
     CUtensorMap mq, mk, mv, mo;
     // (in split mode O is written by the combine kernel; the O map is then unused but valid)
-    if (!make_map(&mq, q, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, k, dt, 2, D, Nk, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, v, dt, 2, D, Nk, bh, 64, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_map(&mq, q, dti, ie, D, N, bh, ib, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, k, dti, ie, D, Nk, bh, ib, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, v, dti, ie, D, Nk, bh, ib, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mo, o, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return FA_ERR_CUDA;
     fa::FwdParams p;
@@ -188,7 +191,8 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.drop = drop;
-    auto kern = fa::fa_fwd_kernel<D, BF16, DROP, SPLIT>;
+    p.out_scale = out_scale;
+    auto kern = fa::fa_fwd_kernel<D, BF16, DROP, SPLIT, F8>;
     static std::atomic<int> smem_done[kMaxDevices];
     cudaError_t e = set_smem(kern, C::SMEM, smem_done, dev);
     if (e != cudaSuccess) {
@@ -564,6 +568,28 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
         return bf16 ? launch_splitkv<64, true>(FA_SPLIT_ARGS) : launch_splitkv<64, false>(FA_SPLIT_ARGS);
     return bf16 ? launch_splitkv<128, true>(FA_SPLIT_ARGS) : launch_splitkv<128, false>(FA_SPLIT_ARGS);
 #undef FA_SPLIT_ARGS
+}
+
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+               int N, int d, float scale, int causal, const int *kv_len, float q_scale,
+               float k_scale, float v_scale, void *stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID_ARG;
+    for (float f : {q_scale, k_scale, v_scale})
+        if (!std::isfinite(f) || !(f > 0.f)) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, N, d, scale, FA_BF16);
+    if (rc != FA_OK) return rc;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    int dev = 0;
+    rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    const SplitOut whole;
+    // the scores see q_scale * k_scale through the softmax scale; V's scale multiplies O
+    return launch_fwd<128, true, false, false, true>(
+        q, k, v, o, lse, B, H, N, N, scale * q_scale * k_scale, causal, kv_len, nullptr, 0,
+        kNoDropout, whole, reinterpret_cast<cudaStream_t>(stream), dev, v_scale);
 }
 
 int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B,

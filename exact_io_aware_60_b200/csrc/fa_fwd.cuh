@@ -46,6 +46,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "dropout.cuh"
 #include "sm100.cuh"
 
@@ -74,6 +76,7 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal;
     DropoutParams drop;  // used by the dropout variant only
+    float out_scale;     // E4M3 variant: V's scale factor, applied to the output
 };
 
 template <int D>
@@ -108,7 +111,47 @@ struct FwdCfg {
     static constexpr uint32_t COL_O = P_OWN ? COL_P + BN / 2 : SBUF * BN;
     static constexpr uint32_t COL_SUM = COL_O + D;      // 16 columns: row sums of 16-bit P
     static constexpr int PV_N = D + 16;                 // O and the row sums in one MMA
+    static constexpr int KS_S = D / 16;                 // MMA K steps of S (32 bytes each)
+    static constexpr int KS_PV = BN / 16;               // MMA K steps of P V
+    static constexpr int PV_STEP = 16 * 128;            // bytes of V rows per P V step
     static_assert(COL_SUM + 16 <= TMEM_COLS, "TMEM budget");
+};
+
+// E4M3 inputs, d = 128: a row of Q, K or V is one 128-byte swizzle block, an MMA step
+// takes K = 32 one-byte elements, and P goes to TMEM as four E4M3 values per column.
+struct FwdCfgF8 {
+    static constexpr int D = 128;
+    static constexpr int BM = 128;
+    static constexpr int BN = 128;
+    static constexpr int HALVES = 1;                    // 128-byte column blocks per row
+    static constexpr int QTILE = BM * 128;
+    static constexpr int QHALF = BM * 128;
+    static constexpr int KTILE = BN * 128;
+    static constexpr int KHALF = BN * 128;
+    static constexpr bool P_OWN = false;
+    static constexpr int SBUF = 2;
+    static constexpr int CTAS_PER_SM = 1;
+    static constexpr int NS = 4;
+    static constexpr int VSTAGE = 2 * KHALF;            // V block + its block of E4M3 ones
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + QTILE;
+    static constexpr int OFF_V = OFF_K + NS * KTILE;
+    static constexpr int OFF_BAR = OFF_V + NS * VSTAGE;
+    static constexpr int USED = OFF_BAR + 256;
+    static constexpr int SLACK = 1024;
+    static constexpr int SMEM = USED + SLACK;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int PBUF = 1;
+    static constexpr uint32_t COL_P = SBUF * BN;
+    static constexpr uint32_t COL_O = SBUF * BN;
+    static constexpr uint32_t COL_SUM = COL_O + D;
+    static constexpr int PV_N = D + 16;
+    static constexpr int KS_S = D / 32;
+    static constexpr int KS_PV = BN / 32;
+    static constexpr int PV_STEP = 32 * 128;
+    static_assert(COL_SUM + 16 <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct FwdBars {
@@ -127,12 +170,15 @@ struct FwdBars {
 // counter-based generator; the normaliser is the fp32 sum of the undropped values).
 // SPLIT: the CTA covers one range of key blocks and writes an fp32 partial output (O
 // normalised by that range's own l) and the range's LSE; a combine kernel merges them.
-template <int D, bool BF16, bool DROP, bool SPLIT>
+// F8: E4M3 Q, K, V (d = 128), kind::f8f6f4 MMAs, P rounded to E4M3 for the P V product,
+// bf16 output (BF16 = true).
+template <int D, bool BF16, bool DROP, bool SPLIT, bool F8 = false>
 __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
               const FwdParams p) {
-    using C = FwdCfg<D>;
+    static_assert(!F8 || (D == 128 && BF16 && !DROP && !SPLIT), "E4M3 variant: d = 128 only");
+    using C = std::conditional_t<F8, FwdCfgF8, FwdCfg<D>>;
     constexpr int BN = C::BN;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -181,7 +227,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     if (warp == 4) {
         // 16-bit ones after every V stage (layout-agnostic: every element is 1)
-        const uint32_t one2 = BF16 ? 0x3F803F80u : 0x3C003C00u;
+        const uint32_t one2 = F8 ? 0x38383838u : (BF16 ? 0x3F803F80u : 0x3C003C00u);
         for (int st = 0; st < C::NS; ++st) {
             uint4 *ones = reinterpret_cast<uint4 *>(sV + st * C::VSTAGE + C::HALVES * C::KHALF);
             for (int i = lane; i < C::KHALF / 16; i += 32) ones[i] = make_uint4(one2, one2, one2, one2);
@@ -242,8 +288,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     } else if (warp == 5) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0 && any_block) {
-            constexpr uint32_t kIdescS = idesc_f16(BF16, false, false, 128, BN);
-            constexpr uint32_t kIdescO = idesc_f16(BF16, false, true, 128, C::PV_N);
+            constexpr uint32_t kIdescS =
+                F8 ? idesc_e4m3(false, false, 128, BN) : idesc_f16(BF16, false, false, 128, BN);
+            constexpr uint32_t kIdescO = F8 ? idesc_e4m3(false, true, 128, C::PV_N)
+                                            : idesc_f16(BF16, false, true, 128, C::PV_N);
             // Descriptors are built once; per k-step and per stage only the 16-byte start
             // address field changes, by compile-time offsets.
             const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
@@ -259,10 +307,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const uint32_t d_tmem = tmem + (uint32_t)((jj % C::SBUF) * BN);
                 const uint64_t kd = k_desc + (uint64_t)((s * C::KTILE) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::KS_S; ++kk) {
                     const uint64_t qo = (uint64_t)(((kk >> 2) * C::QHALF + (kk & 3) * 32) >> 4);
                     const uint64_t ko = (uint64_t)(((kk >> 2) * C::KHALF + (kk & 3) * 32) >> 4);
-                    mma_ss(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
+                    if constexpr (F8) mma_ss_f8(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
+                    else mma_ss(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&bars->s_full[jj % C::SBUF]);
                 return true;
@@ -287,9 +336,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tmem + (C::P_OWN ? C::COL_P : (uint32_t)((jj % C::SBUF) * BN));
                 const uint64_t vd = v_desc + (uint64_t)((s * C::VSTAGE) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts(tmem + C::COL_O, p_tmem + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), kIdescO,
-                           (jj > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < C::KS_PV; ++kk) {
+                    const uint64_t vo = (uint64_t)(kk * C::PV_STEP >> 4);
+                    if constexpr (F8)
+                        mma_ts_f8(tmem + C::COL_O, p_tmem + kk * 8, vd + vo, kIdescO,
+                                  (jj > 0 || kk > 0) ? 1u : 0u);
+                    else
+                        mma_ts(tmem + C::COL_O, p_tmem + kk * 8, vd + vo, kIdescO,
+                               (jj > 0 || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(&bars->kv_empty[s]);
                 mma_commit(&bars->o_full);
                 j = jn;
@@ -353,14 +408,29 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             const float m_use = (m == -INFINITY) ? 0.f : m;
             float sum0 = 0.f, sum1 = 0.f;
-            uint32_t pk[BN / 2];
+            // P in the P V operand format: 16-bit pairs, or (F8) four E4M3 per word
+            constexpr int PW = F8 ? BN / 4 : BN / 2;
+            uint32_t pk[PW];
+            if constexpr (F8) {
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-                const float p0 = ex2(fmaf(s[c], sl2, -m_use));
-                const float p1 = ex2(fmaf(s[c + 1], sl2, -m_use));
-                sum0 += p0;
-                sum1 += p1;
-                pk[c >> 1] = pack2<BF16>(p0, p1);
+                for (int c = 0; c < BN; c += 4) {
+                    const float p0 = ex2(fmaf(s[c], sl2, -m_use));
+                    const float p1 = ex2(fmaf(s[c + 1], sl2, -m_use));
+                    const float p2 = ex2(fmaf(s[c + 2], sl2, -m_use));
+                    const float p3 = ex2(fmaf(s[c + 3], sl2, -m_use));
+                    sum0 += p0 + p2;
+                    sum1 += p1 + p3;
+                    pk[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < BN; c += 2) {
+                    const float p0 = ex2(fmaf(s[c], sl2, -m_use));
+                    const float p1 = ex2(fmaf(s[c + 1], sl2, -m_use));
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[c >> 1] = pack2<BF16>(p0, p1);
+                }
             }
             if constexpr (DROP) {
                 // Keys j*BN + 16u .. +15 of this row: one Philox block each; dropped
@@ -411,7 +481,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             {
                 const uint32_t pb = C::P_OWN ? tmem + lane_base + C::COL_P : sb;
 #pragma unroll
-                for (int h = 0; h < BN / 64; ++h) {
+                for (int h = 0; h < PW / 32; ++h) {
                     uint32_t r[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = pk[h * 32 + i];
@@ -442,6 +512,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float inv;
         if constexpr (DROP) inv = (l > 0.f) ? p.drop.keep_scale / l : 0.f;
         else inv = (l > 0.f && l_round > 0.f) ? 1.f / l_round : 0.f;
+        if constexpr (F8) inv *= p.out_scale;
         const float lse_row = (l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
         if constexpr (SPLIT) {
             // fp32 partial output of this key range, one contiguous row per thread
@@ -466,8 +537,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             if (row < p.N) p.part_lse[prow] = lse_row;
         } else {
+        // O staging: 16-bit [128 x D] in 64-column blocks of 16 KB, over Q (16-bit
+        // inputs) or over the K ring (F8: the E4M3 Q tile is half the size; every K block
+        // has been consumed once the last P V is done).
+        uint8_t *stage = F8 ? sK : sQ;
+        // Warps without query rows leave their staging rows alone: they have not waited
+        // for the tile's MMAs, which may still be reading the staging area (their rows
+        // would fall outside the tensor and be clipped by the store anyway).
 #pragma unroll
-        for (int hf = 0; hf < C::HALVES; ++hf) {
+        for (int hf = 0; hf < (active ? D / 64 : 0); ++hf) {
             uint32_t w[32];
             {
                 uint32_t r[32];
@@ -490,7 +568,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                             __uint_as_float(r[2 * i + 1]) * inv);
             }
             // Row t of this 128-byte column block, 16-byte chunks XOR-swizzled by t % 8.
-            uint8_t *rowp = sQ + hf * C::QHALF + t * 128;
+            uint8_t *rowp = stage + hf * 16384 + t * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint4 v4 = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
@@ -500,8 +578,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (t == 0) {
-            for (int hf = 0; hf < C::HALVES; ++hf)
-                tma_store_3d(&tmO, sQ + hf * C::QHALF, hf * 64, qt * C::BM, bh);
+            for (int hf = 0; hf < D / 64; ++hf)
+                tma_store_3d(&tmO, stage + hf * 16384, hf * 64, qt * C::BM, bh);
             bulk_commit_group();
             bulk_wait_group_read<0>();
         }

@@ -91,6 +91,8 @@ def lib():
             L.fa_fwd_splitkv.restype = i
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, i, i, vp, sz,
                                          vp]
+            L.fa_fwd_fp8.restype = i
+            L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, f, f, f, vp]
             L.fa_bwd_noalloc.restype = i
             L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i,
                                          vp, i, vp]
@@ -343,6 +345,26 @@ def forward_splitkv(q, k, v, *, scale: Optional[float] = None, causal: bool = Fa
     fa_fwd_splitkv(q, k, v, o, lse, scale=scale, causal=causal, kv_len=kv_len,
                    num_splits=num_splits, workspace=ws, stream=stream)
     return o, lse
+
+
+def fa_fwd_fp8(q8, k8, v8, o, lse, *, scale: float, q_scale: float, k_scale: float,
+               v_scale: float, causal: bool = False, kv_len=None, stream=None) -> None:
+    """FP8 forward: q8, k8, v8 are E4M3 tensors (torch.float8_e4m3fn, or their uint8 bytes)
+    [B,H,N,128] with per-tensor scale factors; writes bf16 ``o`` and fp32 ``lse``."""
+    B, H, N, d = q8.shape
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d) \
+                or t.element_size() != 1:
+            raise FAError(FA_ERR_INVALID_ARG, f"{name} must be a contiguous 1-byte CUDA tensor "
+                                              f"of shape {(B, H, N, d)}")
+    _check(o, "o", (B, H, N, d), torch.bfloat16)
+    _check(lse, "lse", (B, H, N), torch.float32)
+    rc = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), o.data_ptr(),
+                          lse.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                          _kv_ptr(kv_len, B), float(q_scale), float(k_scale), float(v_scale),
+                          _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_fp8")
 
 
 def fa_set_timing_events(which: int, start=None, stop=None) -> None:

@@ -192,6 +192,27 @@ FA_API int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, 
                           size_t workspace_bytes, void *stream);
 
 /*
+ * FP8 forward (the FlashAttention-3 low-precision variant the aicassindra page and the
+ * promptingindex page, "Adoption", name): Q, K and V in E4M3 (one byte per element,
+ * [B, H, N, d] like the 16-bit calls), each with one fp32 scale factor, so that the
+ * represented values are q_scale * Q8, k_scale * K8, v_scale * V8.  Computes the same
+ * attention as fa_fwd of those values: S = (scale * q_scale * k_scale) Q8 K8^T in fp32 on
+ * E4M3 tensor cores (kind::f8f6f4), the online softmax in fp32, P rounded to E4M3 for the
+ * P V product (its row sums come out of the same rounded values), O = v_scale * (P V) / l
+ * written in bf16, LSE in fp32.
+ *   q, k, v : DEVICE E4M3 bytes [B, H, N, d]; o: DEVICE bf16 [B, H, N, d]; lse: fp32.
+ *   d       : 128 only (FA_ERR_UNSUPPORTED otherwise).
+ * Accuracy: the inputs are exact (the reference is attention of the scaled E4M3 values);
+ * the rounding of P to E4M3 (3 mantissa bits) perturbs each weight by up to 2^-4
+ * relative, so |O - O_exact| <= 2^-3 max_j |v_j| in the worst case; in practice errors are
+ * far smaller (see the parity tests).  Returns FA_ERR_INVALID_ARG for the fa_fwd checks
+ * or a non-finite / non-positive scale factor.  Forward only (no FP8 backward).
+ */
+FA_API int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                      int H, int N, int d, float scale, int causal, const int *kv_len,
+                      float q_scale, float k_scale, float v_scale, void *stream);
+
+/*
  * Attention with dropout on the probabilities (promptingindex page, "Why attention is
  * memory-bound, not compute-bound": dropout is the op between the softmax and the
  * product with V).  Identical to fa_fwd / fa_bwd except that

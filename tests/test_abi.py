@@ -204,3 +204,24 @@ def call_splitkv(**over):
 ])
 def test_splitkv_rejects_bad_arguments_on_host(over, code):
     assert call_splitkv(**over) == code
+
+
+def call_fp8(**over):
+    a = dict(GOOD, d=128, q=P, k=P, v=P, o=P, lse=P, kv=None, qs=0.5, ks=0.5, vs=0.5)
+    a.update(over)
+    return fa.lib().fa_fwd_fp8(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"],
+                               a["d"], a["scale"], a["causal"], a["kv"], a["qs"], a["ks"],
+                               a["vs"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(v=P + 8), fa.FA_ERR_INVALID_ARG),
+    (dict(qs=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(ks=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(vs=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fp8_rejects_bad_arguments_on_host(over, code):
+    assert call_fp8(**over) == code
