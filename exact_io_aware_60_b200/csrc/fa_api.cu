@@ -173,6 +173,7 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
         !make_map(&mo, o, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return FA_ERR_CUDA;
     fa::FwdParams p;
+    p.o = o;
     p.lse = lse;
     p.kv_len = kv_len;
     p.part_o = so.part_o;
@@ -199,8 +200,13 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
         record_cuda_error(e, "cudaFuncSetAttribute(fwd)");
         return FA_ERR_CUDA;
     }
-    const long long grid = (long long)p.num_q_tiles * so.num_splits * bh;
-    if (grid >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    // Persistent: up to CTAS_PER_SM CTAs per SM walk the (query tile, split, head) items.
+    const long long items = (long long)p.num_q_tiles * so.num_splits * bh;
+    if (items >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+    const long long grid = std::min<long long>(items, (long long)C::CTAS_PER_SM * sms);
     timing_mark(0, 0, st);
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mo, p);
     if (e == cudaSuccess) e = cudaGetLastError();

@@ -54,6 +54,7 @@
 namespace fa {
 
 struct FwdParams {
+    void *o;  // [BH][N][D] 16-bit output (written from registers)
     float *lse;
     const int *kv_len;
     // Split-KV partial outputs (SPLIT only): the normalised O and the LSE of each split's
@@ -156,6 +157,8 @@ struct FwdCfgF8 {
 
 struct FwdBars {
     uint64_t q_full;
+    uint64_t q_empty;  // every S MMA of the current item is done: Q may be reloaded
+    uint64_t o_empty;  // the epilogue has read O: the next item's first P V may start
     uint64_t s_full[2];
     uint64_t s_read;
     uint64_t p_full[2];
@@ -195,28 +198,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: (query tile, key split, head); heaviest causal tiles are launched first.
-    const int bh = blockIdx.x % p.BH;
-    const int rest = blockIdx.x / p.BH;
-    const int split = rest % p.num_splits;
-    const int tile_rank = rest / p.num_splits;
-    const int qt = p.causal ? (p.num_q_tiles - 1 - tile_rank) : tile_rank;
-    const int b = bh / p.H;
-    // Softmax warps that hold at least one query row; the others skip the block loop, and
-    // the per-block barriers count only the active ones.
-    const int n_active = min(4, (p.N - qt * C::BM + 31) >> 5);
-
     if (threadIdx.x == 128) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
-        tma_prefetch_desc(&tmO);
         mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->o_empty, 128);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[i], 32 * n_active);
+            mbar_init(&bars->p_full[i], 128);
         }
-        mbar_init(&bars->s_read, 32 * n_active);
+        mbar_init(&bars->s_read, 128);
         mbar_init(&bars->o_full, 1);
         for (int i = 0; i < C::NS; ++i) {
             mbar_init(&bars->k_full[i], 1);
@@ -226,7 +219,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         fence_mbar_init();
     }
     if (warp == 4) {
-        // 16-bit ones after every V stage (layout-agnostic: every element is 1)
+        // 16-bit (or E4M3) ones after every V stage (layout-agnostic: every element is 1)
         const uint32_t one2 = F8 ? 0x38383838u : (BF16 ? 0x3F803F80u : 0x3C003C00u);
         for (int st = 0; st < C::NS; ++st) {
             uint4 *ones = reinterpret_cast<uint4 *>(sV + st * C::VSTAGE + C::HALVES * C::KHALF);
@@ -241,53 +234,86 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t tmem = bars->tmem_base;
     pdl_wait();  // inputs written by the previous kernel are visible from here on
 
-    int L = p.Nk;
-    if (p.kv_len != nullptr) {
-        L = p.kv_len[b];
-        L = L < 0 ? 0 : (L > p.Nk ? p.Nk : L);
-    }
-    int kv_end = L;
-    if (p.causal) kv_end = min(kv_end, (qt + 1) * C::BM + p.causal_off);
-    int T = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;  // key blocks in range
-    int j_lo = 0;
-    if (p.kv_blocks_per_split > 0) {  // this split's blocks: [j_lo, T)
-        j_lo = split * p.kv_blocks_per_split;
-        T = min(T, j_lo + p.kv_blocks_per_split);
-    }
+    // Persistent CTA: work items are (query tile, key split, head), numbered so that the
+    // heaviest causal tiles come first.  Round r of CTA c takes item r * G + c on even
+    // rounds and r * G + (G - 1 - c) on odd ones (G = grid size).  Every role walks the
+    // same list; key lengths and block masks are read only after the wait above.
+    struct Item {
+        int qt, split, bh, L;
+        int T;            // end of this item's key-block range
+        int j_first;      // first visited key block (T if none)
+        const uint8_t *mrow;
+    };
     // Block-sparse walk: next key block at or after j whose tile is set (T if none).
-    const uint8_t *mrow =
-        p.bmask ? p.bmask + (size_t)bh * p.bmask_bh_stride + (size_t)qt * p.bmask_T : nullptr;
-    auto next_block = [&](int j) -> int {
-        if (mrow)
-            while (j < T && mrow[(j * BN) >> 7] == 0) ++j;
+    auto next_block = [&](const Item &it, int j) -> int {
+        if (it.mrow)
+            while (j < it.T && it.mrow[(j * BN) >> 7] == 0) ++j;
         return j;
     };
-    const int j_first = next_block(j_lo);
-    const bool any_block = j_first < T;
+    auto item_at = [&](int r, Item &it) -> bool {
+        const int G = (int)gridDim.x;
+        const int u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        if (u >= p.num_q_tiles * p.num_splits * p.BH) return false;
+        it.bh = u % p.BH;
+        const int rest = u / p.BH;
+        it.split = rest % p.num_splits;
+        const int tile_rank = rest / p.num_splits;
+        it.qt = p.causal ? (p.num_q_tiles - 1 - tile_rank) : tile_rank;
+        int L = p.Nk;
+        if (p.kv_len != nullptr) {
+            L = p.kv_len[it.bh / p.H];
+            L = L < 0 ? 0 : (L > p.Nk ? p.Nk : L);
+        }
+        it.L = L;
+        int kv_end = L;
+        if (p.causal) kv_end = min(kv_end, (it.qt + 1) * C::BM + p.causal_off);
+        it.T = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;
+        int j_lo = 0;
+        if (p.kv_blocks_per_split > 0) {  // this split's blocks: [j_lo, T)
+            j_lo = it.split * p.kv_blocks_per_split;
+            it.T = min(it.T, j_lo + p.kv_blocks_per_split);
+        }
+        it.mrow = p.bmask ? p.bmask + (size_t)it.bh * p.bmask_bh_stride + (size_t)it.qt * p.bmask_T
+                          : nullptr;
+        it.j_first = next_block(it, j_lo);
+        return true;
+    };
 
     if (warp == 4) {
         // ------------------------------ TMA producer ------------------------------
-        if (lane == 0 && any_block) {
-            mbar_arrive_expect_tx(&bars->q_full, C::QTILE);
-            for (int hf = 0; hf < C::HALVES; ++hf)
-                tma_load_3d(sQ + hf * C::QHALF, &tmQ, &bars->q_full, hf * 64, qt * C::BM, bh);
-            int jj = 0;  // index among the visited blocks: drives stages and phases
-            for (int j = j_first; j < T; j = next_block(j + 1), ++jj) {
-                const int s = jj % C::NS;
-                if (jj >= C::NS && !mbar_wait(&bars->kv_empty[s], ((jj / C::NS) - 1) & 1)) break;
-                mbar_arrive_expect_tx(&bars->k_full[s], C::KTILE);
+        // Q of an item as soon as the previous item's last S MMA is done; K_j / V_j into
+        // the ring, whose stages and phases run on the global block count gj.
+        if (lane == 0) {
+            bool ok = true;
+            int gj = 0, t = 0;  // global block count, items with blocks
+            Item it;
+            for (int r = 0; ok && item_at(r, it); ++r) {
+                if (it.j_first >= it.T) continue;
+                if (t > 0 && !mbar_wait(&bars->q_empty, (t - 1) & 1)) break;
+                mbar_arrive_expect_tx(&bars->q_full, C::QTILE);
                 for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_3d(sK + s * C::KTILE + hf * C::KHALF, &tmK, &bars->k_full[s], hf * 64,
-                                j * BN, bh);
-                mbar_arrive_expect_tx(&bars->v_full[s], C::KTILE);
-                for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_3d(sV + s * C::VSTAGE + hf * C::KHALF, &tmV, &bars->v_full[s], hf * 64,
-                                j * BN, bh);
+                    tma_load_3d(sQ + hf * C::QHALF, &tmQ, &bars->q_full, hf * 64, it.qt * C::BM, it.bh);
+                for (int j = it.j_first; j < it.T; j = next_block(it, j + 1), ++gj) {
+                    const int s = gj % C::NS;
+                    if (gj >= C::NS && !mbar_wait(&bars->kv_empty[s], ((gj / C::NS) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars->k_full[s], C::KTILE);
+                    for (int hf = 0; hf < C::HALVES; ++hf)
+                        tma_load_3d(sK + s * C::KTILE + hf * C::KHALF, &tmK, &bars->k_full[s],
+                                    hf * 64, j * BN, it.bh);
+                    mbar_arrive_expect_tx(&bars->v_full[s], C::KTILE);
+                    for (int hf = 0; hf < C::HALVES; ++hf)
+                        tma_load_3d(sV + s * C::VSTAGE + hf * C::KHALF, &tmV, &bars->v_full[s],
+                                    hf * 64, j * BN, it.bh);
+                }
+                ++t;
             }
         }
     } else if (warp == 5) {
         // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0 && any_block) {
+        if (lane == 0) {
             constexpr uint32_t kIdescS =
                 F8 ? idesc_e4m3(false, false, 128, BN) : idesc_f16(BF16, false, false, 128, BN);
             constexpr uint32_t kIdescO = F8 ? idesc_e4m3(false, true, 128, C::PV_N)
@@ -297,14 +323,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t k_desc = smem_desc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t v_desc = smem_desc_sw128(smem_u32(sV), C::KHALF, 1024);
-            bool ok = mbar_wait(&bars->q_full, 0);
-            tc_fence_after();
-            // jj: index of the visited block (stages, phases and buffers follow it)
-            auto issue_s = [&](int jj) -> bool {
-                const int s = jj % C::NS;
-                if (!mbar_wait(&bars->k_full[s], (jj / C::NS) & 1)) return false;
+            // g: global block index (stages, phases and score buffers follow it)
+            auto issue_s = [&](int g) -> bool {
+                const int s = g % C::NS;
+                if (!mbar_wait(&bars->k_full[s], (g / C::NS) & 1)) return false;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)((jj % C::SBUF) * BN);
+                const uint32_t d_tmem = tmem + (uint32_t)((g % C::SBUF) * BN);
                 const uint64_t kd = k_desc + (uint64_t)((s * C::KTILE) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::KS_S; ++kk) {
@@ -313,65 +337,95 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if constexpr (F8) mma_ss_f8(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
                     else mma_ss(d_tmem, q_desc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full[jj % C::SBUF]);
+                mma_commit(&bars->s_full[g % C::SBUF]);
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            int jj = 0;
-            for (int j = j_first; ok && j < T; ++jj) {
-                const int jn = next_block(j + 1);
-                if (jn < T) {
-                    if (C::P_OWN) {
-                        // S_{jj+1} overwrites S_jj as soon as the softmax has read it.
-                        if (!mbar_wait(&bars->s_read, jj & 1) || !issue_s(jj + 1)) break;
-                    } else if (C::SBUF == 2) {
-                        if (!issue_s(jj + 1)) break;  // the other score buffer is free
-                    }
-                }
-                const int s = jj % C::NS;
-                if (!mbar_wait(&bars->p_full[jj % C::SBUF], (jj / C::SBUF) & 1)) break;
-                if (!mbar_wait(&bars->v_full[s], (jj / C::NS) & 1)) break;
+            bool ok = true;
+            int gj = 0, t = 0;
+            Item it;
+            for (int r = 0; ok && item_at(r, it); ++r) {
+                if (it.j_first >= it.T) continue;
+                if (!mbar_wait(&bars->q_full, t & 1)) break;
                 tc_fence_after();
-                const uint32_t p_tmem =
-                    tmem + (C::P_OWN ? C::COL_P : (uint32_t)((jj % C::SBUF) * BN));
-                const uint64_t vd = v_desc + (uint64_t)((s * C::VSTAGE) >> 4);
+                // The item's first S overwrites the previous block's S once the softmax has
+                // read it (d = 64); at d = 128 its buffer held P_{g-2}, consumed by an
+                // earlier P V.
+                if (C::P_OWN && gj > 0 && !mbar_wait(&bars->s_read, (gj - 1) & 1)) break;
+                if (!issue_s(gj)) break;
+                int jj = 0;
+                for (int j = it.j_first; j < it.T; ++jj) {
+                    const int g = gj + jj;
+                    const int jn = next_block(it, j + 1);
+                    if (jn < it.T) {
+                        if (C::P_OWN) {
+                            // S_{g+1} overwrites S_g as soon as the softmax has read it.
+                            if (!mbar_wait(&bars->s_read, g & 1) || !issue_s(g + 1)) { ok = false; break; }
+                        } else if (C::SBUF == 2) {
+                            if (!issue_s(g + 1)) { ok = false; break; }  // other buffer is free
+                        }
+                    } else {
+                        mma_commit(&bars->q_empty);  // every S of the item is issued: Q is free
+                    }
+                    const int s = g % C::NS;
+                    if (!mbar_wait(&bars->p_full[g % C::SBUF], (g / C::SBUF) & 1) ||
+                        !mbar_wait(&bars->v_full[s], (g / C::NS) & 1)) { ok = false; break; }
+                    // the item's first P V restarts O: the previous epilogue must have read it
+                    if (jj == 0 && t > 0 && !mbar_wait(&bars->o_empty, (t - 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t p_tmem =
+                        tmem + (C::P_OWN ? C::COL_P : (uint32_t)((g % C::SBUF) * BN));
+                    const uint64_t vd = v_desc + (uint64_t)((s * C::VSTAGE) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < C::KS_PV; ++kk) {
-                    const uint64_t vo = (uint64_t)(kk * C::PV_STEP >> 4);
-                    if constexpr (F8)
-                        mma_ts_f8(tmem + C::COL_O, p_tmem + kk * 8, vd + vo, kIdescO,
-                                  (jj > 0 || kk > 0) ? 1u : 0u);
-                    else
-                        mma_ts(tmem + C::COL_O, p_tmem + kk * 8, vd + vo, kIdescO,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < C::KS_PV; ++kk) {
+                        const uint64_t vo = (uint64_t)(kk * C::PV_STEP >> 4);
+                        if constexpr (F8)
+                            mma_ts_f8(tmem + C::COL_O, p_tmem + kk * 8, vd + vo, kIdescO,
+                                      (jj > 0 || kk > 0) ? 1u : 0u);
+                        else
+                            mma_ts(tmem + C::COL_O, p_tmem + kk * 8, vd + vo, kIdescO,
+                                   (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars->kv_empty[s]);
+                    mma_commit(&bars->o_full);
+                    j = jn;
                 }
-                mma_commit(&bars->kv_empty[s]);
-                mma_commit(&bars->o_full);
-                j = jn;
+                gj += jj;
+                ++t;
             }
         }
     } else {
         // ------------------------------ softmax warps ------------------------------
         const int t = threadIdx.x;  // 0..127: row in the tile and TMEM lane
-        const int row = qt * C::BM + t;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t ob = tmem + lane_base + C::COL_O;
         const float sl2 = p.scale_log2;
+        bool ok = true;
+        int gj = 0;  // global block count
+        Item it;
+        for (int r = 0; item_at(r, it); ++r) {
+        const int qt = it.qt, bh = it.bh, L = it.L, T = it.T, split = it.split;
+        const int row = qt * C::BM + t;
+        const bool any_block = it.j_first < T;
         float m = -INFINITY;  // running max, in units of log2 (already scaled)
         float l = 0.f;        // running normaliser
-        bool ok = true;
-        int jj = 0;  // visited blocks so far
-        const bool active = warp < n_active;
-        for (int j = active ? j_first : T; j < T; j = next_block(j + 1), ++jj) {
-            if (!mbar_wait(&bars->s_full[jj % C::SBUF], (jj / C::SBUF) & 1)) { ok = false; break; }
+        int jj = 0;           // blocks of this item so far
+        for (int j = it.j_first; ok && j < T; j = next_block(it, j + 1), ++jj) {
+            const int g = gj + jj;
+            // (waits are voted on, so that a warp leaves the loop together: the loop body
+            // has warp-wide TMEM loads and votes)
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[g % C::SBUF], (g / C::SBUF) & 1))) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            const uint32_t sb = tmem + lane_base + (uint32_t)((jj % C::SBUF) * BN);
+            const uint32_t sb = tmem + lane_base + (uint32_t)((g % C::SBUF) * BN);
             float s[BN];
             {
-                uint32_t r[BN];
-                if constexpr (BN == 64) tmem_ld64(sb, r);
-                else tmem_ld128(sb, r);
+                uint32_t rr[BN];
+                if constexpr (BN == 64) tmem_ld64(sb, rr);
+                else tmem_ld128(sb, rr);
 #pragma unroll
-                for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(rr[i]);
             }
             if (C::P_OWN) {
                 tc_fence_before();
@@ -438,9 +492,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const uint32_t g0 = (uint32_t)(j * BN) >> 4;
 #pragma unroll
                 for (int u = 0; u < BN / 16; ++u) {
-                    const uint4 r = philox4x32_10(g0 + u, (uint32_t)row, (uint32_t)bh,
-                                                  p.drop.offset, p.drop.seed_lo, p.drop.seed_hi);
-                    const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+                    const uint4 rr = philox4x32_10(g0 + u, (uint32_t)row, (uint32_t)bh,
+                                                   p.drop.offset, p.drop.seed_lo, p.drop.seed_hi);
+                    const uint32_t w4[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         uint32_t m01, m23;
@@ -451,60 +505,62 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
             }
             l = l * alpha + (sum0 + sum1);
-            // Every phase of o_full is waited on, in order, so that a parity wait can
-            // never alias a phase two ahead.  P_{j-1} V_{j-1} was issued a whole softmax
-            // block ago, so this wait is normally already satisfied.  It also frees P's
-            // columns (d = 64) before P_j is written there.
-            if (jj > 0) {
-                if (!mbar_wait(&bars->o_full, (jj - 1) & 1)) { ok = false; break; }
+            // Every phase of o_full is waited on, in order, so that a parity wait can never
+            // alias a phase two ahead.  P_{g-1} V_{g-1} (possibly the previous item's last)
+            // was issued a whole softmax block ago, so this wait is normally satisfied.  It
+            // also frees P's columns (d = 64) before P_g is written there.
+            if (g > 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full, (g - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
             }
             if (jj > 0 && any_grow) {
-                // Rescale the accumulated output and row sums (P_{j-1} V_{j-1} is done).
-                const uint32_t ob = tmem + lane_base + C::COL_O;
+                // Rescale the accumulated output and row sums (P_{g-1} V_{g-1} is done).
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(ob + c * 32, r);
+                    uint32_t rr[32];
+                    tmem_ld32(ob + c * 32, rr);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(ob + c * 32, r);
+                    for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+                    tmem_st32(ob + c * 32, rr);
                 }
                 {
-                    uint32_t r[16];
-                    tmem_ld16(ob + D, r);
+                    uint32_t rr[16];
+                    tmem_ld16(ob + D, rr);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st16(ob + D, r);
+                    for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+                    tmem_st16(ob + D, rr);
                 }
             }
             {
                 const uint32_t pb = C::P_OWN ? tmem + lane_base + C::COL_P : sb;
 #pragma unroll
                 for (int h = 0; h < PW / 32; ++h) {
-                    uint32_t r[32];
+                    uint32_t rr[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = pk[h * 32 + i];
-                    tmem_st32(pb + h * 32, r);
+                    for (int i = 0; i < 32; ++i) rr[i] = pk[h * 32 + i];
+                    tmem_st32(pb + h * 32, rr);
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->p_full[jj % C::SBUF]);
+            mbar_arrive(&bars->p_full[g % C::SBUF]);
         }
 
-        // ------------------------------ epilogue ------------------------------
-        pdl_launch_dependents();
+        // ------------------------------ epilogue of the item ---------------------------
+        Item nxt;
+        if (!item_at(r + 1, nxt)) pdl_launch_dependents();  // this CTA's last item
         if (ok && jj > 0) {
-            ok = mbar_wait(&bars->o_full, (jj - 1) & 1);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, (gj + jj - 1) & 1));
             tc_fence_after();
         }
-        const uint32_t ob = tmem + lane_base + C::COL_O;
-        const bool have = active && any_block;  // warp-uniform: TMEM loads are warp-wide
+        const bool have = any_block;  // warp-uniform: TMEM loads are warp-wide
         float l_round = 0.f;
         if (have) {
-            uint32_t r[16];
-            tmem_ld16(ob + D, r);
-            l_round = __uint_as_float(r[0]);
+            uint32_t rr[16];
+            tmem_ld16(ob + D, rr);
+            l_round = __uint_as_float(rr[0]);
         }
         // Without dropout the output is divided by the sum of the rounded probabilities
         // the MMA used; with dropout those no longer sum the row, and the output is
@@ -514,77 +570,50 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         else inv = (l > 0.f && l_round > 0.f) ? 1.f / l_round : 0.f;
         if constexpr (F8) inv *= p.out_scale;
         const float lse_row = (l > 0.f) ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
-        if constexpr (SPLIT) {
-            // fp32 partial output of this key range, one contiguous row per thread
-            const size_t prow = ((size_t)split * p.BH + bh) * p.N + row;
-            float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * D);
+        // O straight from TMEM to registers to global memory, 32 columns at a time; the
+        // accumulator is released (o_empty) once every column has been read.
 #pragma unroll
-            for (int c32 = 0; c32 < D / 32; ++c32) {
-                uint32_t r[32];
-                if (have) {
-                    tmem_ld32(ob + c32 * 32, r);
-                } else {
+        for (int c32 = 0; c32 < D / 32; ++c32) {
+            uint32_t rr[32];
+            if (have) {
+                tmem_ld32(ob + c32 * 32, rr);
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = 0u;
-                }
-                if (row < p.N) {
+                for (int i = 0; i < 32; ++i) rr[i] = 0u;
+            }
+            if (c32 == D / 32 - 1 && any_block) {
+                tc_fence_before();
+                mbar_arrive(&bars->o_empty);
+            }
+            if (row < p.N) {
+                if constexpr (SPLIT) {
+                    const size_t prow = ((size_t)split * p.BH + bh) * p.N + row;
+                    float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * D) + c32 * 8;
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        dst[c32 * 8 + i] = make_float4(
-                            __uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                            __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
-                }
-            }
-            if (row < p.N) p.part_lse[prow] = lse_row;
-        } else {
-        // O staging: 16-bit [128 x D] in 64-column blocks of 16 KB, over Q (16-bit
-        // inputs) or over the K ring (F8: the E4M3 Q tile is half the size; every K block
-        // has been consumed once the last P V is done).
-        uint8_t *stage = F8 ? sK : sQ;
-        // Warps without query rows leave their staging rows alone: they have not waited
-        // for the tile's MMAs, which may still be reading the staging area (their rows
-        // would fall outside the tensor and be clipped by the store anyway).
-#pragma unroll
-        for (int hf = 0; hf < (active ? D / 64 : 0); ++hf) {
-            uint32_t w[32];
-            {
-                uint32_t r[32];
-                if (have) {
-                    tmem_ld32(ob + hf * 64, r);
+                        dst[i] = make_float4(
+                            __uint_as_float(rr[4 * i]) * inv, __uint_as_float(rr[4 * i + 1]) * inv,
+                            __uint_as_float(rr[4 * i + 2]) * inv, __uint_as_float(rr[4 * i + 3]) * inv);
                 } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) +
+                                                           ((size_t)bh * p.N + row) * D) + c32 * 4;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[q4] = make_uint4(
+                            pack2<BF16>(__uint_as_float(rr[8 * q4]) * inv, __uint_as_float(rr[8 * q4 + 1]) * inv),
+                            pack2<BF16>(__uint_as_float(rr[8 * q4 + 2]) * inv, __uint_as_float(rr[8 * q4 + 3]) * inv),
+                            pack2<BF16>(__uint_as_float(rr[8 * q4 + 4]) * inv, __uint_as_float(rr[8 * q4 + 5]) * inv),
+                            pack2<BF16>(__uint_as_float(rr[8 * q4 + 6]) * inv, __uint_as_float(rr[8 * q4 + 7]) * inv));
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv,
-                                       __uint_as_float(r[2 * i + 1]) * inv);
-                if (have) {
-                    tmem_ld32(ob + hf * 64 + 32, r);
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[16 + i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv,
-                                            __uint_as_float(r[2 * i + 1]) * inv);
-            }
-            // Row t of this 128-byte column block, 16-byte chunks XOR-swizzled by t % 8.
-            uint8_t *rowp = stage + hf * 16384 + t * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v4 = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-                *reinterpret_cast<uint4 *>(rowp + ((c ^ (t & 7)) << 4)) = v4;
             }
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (t == 0) {
-            for (int hf = 0; hf < D / 64; ++hf)
-                tma_store_3d(&tmO, stage + hf * 16384, hf * 64, qt * C::BM, bh);
-            bulk_commit_group();
-            bulk_wait_group_read<0>();
+        if (row < p.N) {
+            if constexpr (SPLIT) p.part_lse[((size_t)split * p.BH + bh) * p.N + row] = lse_row;
+            else p.lse[(size_t)bh * p.N + row] = lse_row;
         }
-        if (row < p.N) p.lse[(size_t)bh * p.N + row] = lse_row;
-        }  // !SPLIT
+        if (any_block) gj += jj;
+        if (!ok) break;
+        }  // items
     }
 
     tc_fence_before();
