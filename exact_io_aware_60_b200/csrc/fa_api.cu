@@ -165,12 +165,10 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     const CUtensorMapDataType dti = F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : dt;
     const int ie = F8 ? 1 : 2, ib = F8 ? 128 : 64;
     const long long bh = (long long)B * H;
-    CUtensorMap mq, mk, mv, mo;
-    // (in split mode O is written by the combine kernel; the O map is then unused but valid)
+    CUtensorMap mq, mk, mv;  // O is written from registers (or, split-KV, by the combine)
     if (!make_map(&mq, q, dti, ie, D, N, bh, ib, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mk, k, dti, ie, D, Nk, bh, ib, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, v, dti, ie, D, Nk, bh, ib, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mo, o, dt, 2, D, N, bh, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map(&mv, v, dti, ie, D, Nk, bh, ib, C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return FA_ERR_CUDA;
     fa::FwdParams p;
     p.o = o;
@@ -208,7 +206,7 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
         sms = 148;
     const long long grid = std::min<long long>(items, (long long)C::CTAS_PER_SM * sms);
     timing_mark(0, 0, st);
-    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mo, p);
+    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, p);
     if (e == cudaSuccess) e = cudaGetLastError();
     timing_mark(0, 1, st);
     if (e != cudaSuccess) {

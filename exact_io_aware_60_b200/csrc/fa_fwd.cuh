@@ -7,9 +7,12 @@
 // maximum m and normaliser l, rescaling the accumulated output whenever m grows.  Only
 // O and the row statistics leave the chip; the N x N score matrix never exists in HBM.
 //
-// B200 mapping (one CTA = one 128-row query tile of one (batch, head)):
-//   warp 4      TMA producer: Q once, then K_j / V_j into an NS-stage shared-memory ring
-//               (128-byte swizzle, mbarrier transaction counts).
+// B200 mapping: persistent CTAs (two per SM at d = 64), each walking a static list of
+// work items = 128-row query tiles of one (batch, head) (and one key range in split-KV
+// mode).  Per CTA:
+//   warp 4      TMA producer: Q of an item once the previous item's last S MMA is done,
+//               then K_j / V_j into an NS-stage shared-memory ring (128-byte swizzle,
+//               mbarrier transaction counts) that runs on across items.
 //   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM, then O += P_j V_j with
 //               P_j read straight from TMEM.
 //   warps 0..3  softmax, one query row per thread (TMEM lane = row): load S_j, mask on
@@ -17,8 +20,8 @@
 //               MUFU ex2, row sum, P_j written back into TMEM as 16-bit pairs.
 //               The output rescale is lazy: m only moves when the row max grows by more
 //               than 2^8, which leaves the result exact because O and l always share the
-//               same m.  Epilogue: O / l' -> 16-bit, staged swizzled in shared memory and
-//               written with one TMA store; LSE = ln2 * (m + log2 l).
+//               same m.  Epilogue: O / l' -> 16-bit, written from registers row by row
+//               (no staging, so the next item's Q can load early); LSE = ln2 * (m + log2 l).
 //   Normaliser: the tensor core multiplies V by P rounded to 16 bits, so the output is
 //   divided by l' = sum of exactly those rounded values, produced by the same PV MMA
 //   (its B operand carries 16 extra columns of ones after V) in 16 extra TMEM columns.
@@ -178,8 +181,7 @@ struct FwdBars {
 template <int D, bool BF16, bool DROP, bool SPLIT, bool F8 = false>
 __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-              const FwdParams p) {
+              const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     static_assert(!F8 || (D == 128 && BF16 && !DROP && !SPLIT), "E4M3 variant: d = 128 only");
     using C = std::conditional_t<F8, FwdCfgF8, FwdCfg<D>>;
     constexpr int BN = C::BN;
