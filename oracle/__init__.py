@@ -88,6 +88,8 @@ def _load():
                                                 ctypes.c_void_p]
             lib.oracle_threads.restype = ctypes.c_int
             lib.oracle_threads.argtypes = []
+            lib.oracle_set_threads.restype = None
+            lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -95,6 +97,12 @@ def _load():
 def threads() -> int:
     """OpenMP threads the oracle uses."""
     return int(_load().oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """OpenMP threads for later oracle calls (timing only; results do not depend on it
+    beyond the order of the dK/dV sums)."""
+    _load().oracle_set_threads(int(n))
 
 
 def dropout_threshold(p) -> int:

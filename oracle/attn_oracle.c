@@ -165,6 +165,16 @@ int oracle_threads(void)
 #endif
 }
 
+/* Sets the OpenMP thread count of later calls (for timing the oracle on fewer cores). */
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /*
  * Exact attention for the query rows rows[0..R) of one (batch, head).
  *
