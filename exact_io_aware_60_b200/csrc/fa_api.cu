@@ -398,11 +398,25 @@ int resolve_splits(long long BH, int Nq, int Nk, int d, int requested, int sms, 
     if (requested > 0) {
         splits = std::min(requested, kblocks);
     } else {
+        // The split count that finishes first on a persistent grid of `slots` CTAs:
+        // (query tile, split, head) items of bps key blocks each are dealt out in rounds
+        // of `slots`; a round costs its blocks plus about two blocks' worth of per-item
+        // work (the Q tile, the fp32 partial output).  Splits of fewer than two blocks,
+        // and more than 128 splits, are not considered.
         const long long tiles = (long long)((Nq + 127) / 128) * BH;
         const long long slots = (long long)sms * (d == 64 ? 2 : 1);
-        const long long want = (2 * slots + tiles - 1) / tiles;
-        splits = (int)std::min<long long>(want, std::max(1, kblocks / 2));
-        splits = std::max(1, std::min(splits, 128));
+        const int max_s = std::max(1, std::min(128, kblocks / 2));
+        long long best = -1;
+        splits = 1;
+        for (int sp = 1; sp <= max_s; ++sp) {
+            const int b = (kblocks + sp - 1) / sp;
+            const long long items = tiles * ((kblocks + b - 1) / b);
+            const long long cost = ((items + slots - 1) / slots) * (b + 2);
+            if (best < 0 || cost < best) {
+                best = cost;
+                splits = sp;
+            }
+        }
     }
     const int bps = (kblocks + splits - 1) / splits;
     *blocks_per = bps;

@@ -171,9 +171,10 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
  * it is fa_fwd).
  *   q, o       : DEVICE [B, H, Nq, d] 16-bit; lse: DEVICE [B, H, Nq] fp32.
  *   k, v       : DEVICE [B, H, Nk, d] 16-bit.
- *   num_splits : 0 = chosen by the library (about two waves of CTAs, at least two key
- *                blocks per split), else 1 .. FA_MAX_SPLITS (capped by the number of key
- *                blocks: 64 keys at d = 64, 128 at d = 128).
+ *   num_splits : 0 = chosen by the library (the count, up to 128 with at least two key
+ *                blocks per split, that minimises rounds x (blocks per split + 2) on a
+ *                grid of one persistent CTA per SM slot), else 1 .. FA_MAX_SPLITS (capped
+ *                by the number of key blocks: 64 keys at d = 64, 128 at d = 128).
  *   workspace  : DEVICE scratch of fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d,
  *                num_splits) bytes, 256-byte aligned, owned by the caller (may be NULL when
  *                that size is 0, i.e. when the call resolves to one split).  The size is

@@ -183,6 +183,31 @@ def test_splitkv_workspace_bytes():
     assert L.fa_fwd_splitkv_workspace_bytes(1, 1, 1, 100, 64, 10000) == 0
 
 
+def _auto_splits(B, H, Nq, Nk, d):
+    """Split count behind the automatic workspace size (1 when none is needed)."""
+    r256 = lambda x: ((x + 255) // 256) * 256
+    n = fa.lib().fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, 0)
+    if n == 0:
+        return 1
+    found = [sp for sp in range(2, 129) if r256(sp * B * H * Nq * d * 4) + r256(sp * B * H * Nq * 4) == n]
+    assert len(found) == 1, (n, found)
+    return found[0]
+
+
+def test_splitkv_automatic_split_count():
+    # decode (one query tile per head, fewer tiles than SMs): the keys are split, into
+    # pieces of at least two key blocks, and never more than 128 of them
+    for B, H, Nk, d in ((8, 16, 32768, 128), (1, 8, 131072, 64), (2, 2, 5000, 64)):
+        sp = _auto_splits(B, H, 1, Nk, d)
+        bn = 64 if d == 64 else 128
+        kblocks = -(-Nk // bn)
+        assert 1 < sp <= 128 and -(-kblocks // sp) >= 2, (B, H, Nk, d, sp)
+    # many query tiles per SM already: no split
+    assert _auto_splits(64, 32, 512, 4096, 64) == 1
+    # too few key blocks to split
+    assert _auto_splits(1, 1, 1, 200, 128) == 1
+
+
 def call_splitkv(**over):
     a = dict(GOOD, Nq=4, Nk=64, q=P, k=P, v=P, o=P, lse=P, kv=None, splits=0, ws=P,
              ws_bytes=1 << 30)
