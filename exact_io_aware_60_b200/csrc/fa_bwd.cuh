@@ -13,18 +13,23 @@
 // Three kernels, all on the caller's stream:
 //   1. fa_bwd_prep_kernel: D_i = rowsum(dO o O) in fp32, LSE in base 2 (padded to whole
 //      128-row tiles, +inf where there is no row), and zeroes the fp32 dQ accumulator.
-//   2. fa_bwd_kernel: one CTA per 128-key tile of one (batch, head), looping over the
-//      128-query tiles that can see it (causal: only tiles on or below the diagonal).
-//        warp 8      TMA producer: K, V once; Q_i, dO_i (+ LSE_i, D_i) into a 2/3-stage ring.
-//        warp 5      MMA issuer (one thread), all on tcgen05 with fp32 TMEM accumulators:
+//   2. fa_bwd_kernel: persistent CTAs (one per SM) walking (128-key tile, head) items, each
+//      looping over the 128-query tiles that can see its keys (causal: only tiles on or
+//      below the diagonal).
+//        warp 8      TMA producer: K, V once per item; Q_i, dO_i (+ LSE_i, D_i) into a
+//                    2/3-stage ring.
+//        warp 9      MMA issuer (one thread), all on tcgen05 with fp32 TMEM accumulators:
 //                    S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i, dK += dS^T Q_i
 //                    (P^T, dS^T read from TMEM), dQ_i = dS K (dS from shared memory).
-//        warps 0..3  one key row per thread: P^T = 2^(S^T scale log2e - LSE2), written back
-//                    to TMEM as 16-bit pairs; dS^T = P^T o (dP^T - D) to TMEM and, in the
-//                    transposed operand layout, to shared memory; epilogue writes dK, dV.
-//        warps 6..9  drain dQ_i from TMEM and add it into the fp32 accumulator in global
-//                    memory (TMA reduce-add of a swizzled staging tile for d = 64; vector
-//                    red.global.add for d = 128, where shared memory is fully used).
+//        warps 0..7  one key row per thread and half of the query columns per warp
+//                    (lane quarter w % 4, query half w / 4): P^T = 2^(S^T scale log2e -
+//                    LSE2), written back to TMEM as 16-bit pairs; dS^T = P^T o (dP^T - D)
+//                    to TMEM and, in the transposed operand layout, to shared memory;
+//                    the item's epilogue writes dK, dV.
+//        warps 10..13 drain dQ_i from TMEM through a swizzled shared-memory staging tile
+//                    and a TMA reduce-add into the fp32 accumulator in global memory (own
+//                    staging area at d = 64; at d = 128, where shared memory is full, the
+//                    dS buffer in two 64-column rounds, free between the dQ MMA and dS_{i+1}).
 //   3. fa_bwd_convert_kernel: dQ = scale * dQ_acc in the input dtype.
 #pragma once
 
@@ -151,7 +156,10 @@ struct BwdCfg {
     static constexpr int TILE = 128 * D * 2;  // one 128-row tile of Q / K / V / dO
     static constexpr int HALF = 128 * 128;    // one 128-byte column block of a tile
     static constexpr int HALVES = D / 64;
-    static constexpr bool DQ_TMA = (D == 64);  // dQ drain by TMA reduce (else red.v4)
+    // dQ leaves TMEM through a shared-memory staging area and a TMA reduce-add: its own
+    // 32 KB at d = 64; at d = 128 (no room) the dS buffer, 64 columns at a time, which is
+    // free between the dQ MMA that reads dS_i and the P/dS warps' writing of dS_{i+1}.
+    static constexpr bool DQ_IN_DS = (D == 128);
     // d = 64: P^T gets its own TMEM columns, so S_{i+1} can overwrite S_i as soon as it
     // has been read.  d = 128: TMEM is full; P^T overwrites S^T and S_{i+1} waits for dV_i.
     static constexpr bool P_OWN = (D == 64);
@@ -165,7 +173,7 @@ struct BwdCfg {
     static constexpr int OFF_DO = OFF_Q + QS * TILE;  // QS stages
     static constexpr int OFF_DS = OFF_DO + QS * TILE; // 128 x 128 16-bit, operand layout
     static constexpr int OFF_DQ = OFF_DS + 32768;    // fp32 staging (d = 64 only)
-    static constexpr int DQ_BYTES = DQ_TMA ? 128 * D * 4 : 0;
+    static constexpr int DQ_BYTES = DQ_IN_DS ? 0 : 128 * D * 4;
     static constexpr int OFF_LSE = OFF_DQ + DQ_BYTES;  // QS x 512 B
     static constexpr int OFF_DV = OFF_LSE + QS * 512;  // QS x 512 B
     static constexpr int OFF_BAR = OFF_DV + QS * 512;
@@ -195,6 +203,7 @@ struct BwdBars {
     uint64_t q_full[3];
     uint64_t do_full[3];
     uint64_t stage_empty[3];
+    uint64_t dq_stage_free;  // d = 128: the dQ drain has finished with the dS buffer
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
         dkv_full, dkv_empty;
     uint32_t tmem_base;
@@ -243,7 +252,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tma_prefetch_desc(&tmdO);
         tma_prefetch_desc(&tmdK);
         tma_prefetch_desc(&tmdV);
-        if (C::DQ_TMA) tma_prefetch_desc(&tmdQacc);
+        tma_prefetch_desc(&tmdQacc);
         mbar_init(&bars->kv_full, 1);
         for (int i = 0; i < C::QS; ++i) {
             mbar_init(&bars->q_full[i], 1);
@@ -259,6 +268,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bars->ds_empty, 1);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 128);
+        mbar_init(&bars->dq_stage_free, 1);
         mbar_init(&bars->dkv_full, 1);
         mbar_init(&bars->dkv_empty, 256);
         fence_mbar_init();
@@ -478,54 +488,46 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int i = 0, qi = it.q_first; i < it.n; ++i, qi = next_q(it, qi + 1)) {
             if (!mbar_wait(&bars->dq_full, (gi + i) & 1)) { ok = false; break; }
             tc_fence_after();
-            if constexpr (C::DQ_TMA) {
-                if (gt == 0) bulk_wait_group_read<0>();
-                named_bar_sync(2, 128);
-                // D/32 boxes of [128 rows][32 fp32], 16-byte chunks swizzled by row % 8.
+            // Boxes of [128 rows][32 fp32], 16-byte chunks swizzled by row % 8, staged
+            // ROUND_BOXES at a time (all D/32 at d = 64; two per round in the dS buffer at
+            // d = 128), each round handed to a TMA reduce-add into the fp32 accumulator.
+            constexpr int ROUND_BOXES = C::DQ_IN_DS ? 2 : D / 32;
+            uint8_t *stage = C::DQ_IN_DS ? sdS : sDQ;
 #pragma unroll
-                for (int bx = 0; bx < D / 32; ++bx) {
+            for (int b0 = 0; b0 < D / 32; b0 += ROUND_BOXES) {
+                if (gt == 0) bulk_wait_group_read<0>();  // the previous reduce has read it
+                named_bar_sync(2, 128);
+#pragma unroll
+                for (int bx = 0; bx < ROUND_BOXES; ++bx) {
                     uint32_t w[32];
-                    tmem_ld32(tmem + lane_base + C::COL_DQ + bx * 32, w);
-                    uint8_t *rowp = sDQ + bx * 16384 + r * 128;
+                    tmem_ld32(tmem + lane_base + C::COL_DQ + (b0 + bx) * 32, w);
+                    uint8_t *rowp = stage + bx * 16384 + r * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         *reinterpret_cast<uint4 *>(rowp + ((c ^ (r & 7)) << 4)) =
                             make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
                 }
-                tc_fence_before();
-                mbar_arrive(&bars->dq_empty);
+                if (b0 + ROUND_BOXES == D / 32) {  // every dQ column is out of TMEM
+                    tc_fence_before();
+                    mbar_arrive(&bars->dq_empty);
+                }
                 fence_proxy_async_smem();
                 named_bar_sync(2, 128);
                 if (gt == 0) {
 #pragma unroll
-                    for (int bx = 0; bx < D / 32; ++bx)
-                        tma_reduce_add_3d(&tmdQacc, sDQ + bx * 16384, bx * 32, qi * 128, bh);
+                    for (int bx = 0; bx < ROUND_BOXES; ++bx)
+                        tma_reduce_add_3d(&tmdQacc, stage + bx * 16384, (b0 + bx) * 32, qi * 128, bh);
                     bulk_commit_group();
                 }
-            } else {
-                const int row = qi * 128 + r;
-                float *dst = p.dq_acc + ((size_t)bh * p.N + (row < p.N ? row : 0)) * D;
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t w[32];
-                    tmem_ld32(tmem + lane_base + C::COL_DQ + c * 32, w);
-                    if (row < p.N) {
-#pragma unroll
-                        for (int k = 0; k < 32; k += 4)
-                            red_add_v4(dst + c * 32 + k, __uint_as_float(w[k]),
-                                       __uint_as_float(w[k + 1]), __uint_as_float(w[k + 2]),
-                                       __uint_as_float(w[k + 3]));
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&bars->dq_empty);
+            }
+            if (C::DQ_IN_DS && gt == 0) {
+                bulk_wait_group_read<0>();  // the dS buffer may take dS_{i+1}
+                mbar_arrive(&bars->dq_stage_free);
             }
         }
         gi += it.n;
         }
-        if constexpr (C::DQ_TMA) {
-            if (gt == 0) bulk_wait_group<0>();
-        }
+        if (gt == 0) bulk_wait_group<0>();
     } else {
         // ------------------------------ P / dS warps ------------------------------
         const int quarter = warp & 3;
@@ -630,7 +632,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_arrive(&bars->p_full);
 
             if (!mbar_wait(&bars->dp_full, g & 1) || !mbar_wait(&bars->do_full[s], (g / C::QS) & 1) ||
-                (g > 0 && !mbar_wait(&bars->ds_empty, (g - 1) & 1))) {
+                (g > 0 && !mbar_wait(&bars->ds_empty, (g - 1) & 1)) ||
+                // d = 128: the dQ drain has staged dQ_{g-1} through the dS buffer and let go
+                (C::DQ_IN_DS && g > 0 && !mbar_wait(&bars->dq_stage_free, (g - 1) & 1))) {
                 ok = false;
                 break;
             }
@@ -680,7 +684,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         Item nxt;
         if (!item_at(rr + 1, nxt)) pdl_launch_dependents();  // this CTA's last item
         if (ok && n > 0) {
-            ok = mbar_wait(&bars->dkv_full, tn & 1);
+            ok = mbar_wait(&bars->dkv_full, tn & 1) &&
+                 // d = 128: the dQ drain of the item's last iteration is done with the dS buffer
+                 (!C::DQ_IN_DS || mbar_wait(&bars->dq_stage_free, (gi + n - 1) & 1));
             tc_fence_after();
         }
         // Staging in the dS buffer (free: every MMA of the item is done; 32 KB): both

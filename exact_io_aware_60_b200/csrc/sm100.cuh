@@ -481,13 +481,6 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
         : "memory");
 }
 
-// Vector fp32 reduction into global memory (performed at L2, no return value).
-__device__ __forceinline__ void red_add_v4(float *gaddr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gaddr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
-
 // ----------------------------------------------------------------------------------
 // small numeric helpers
 // ----------------------------------------------------------------------------------
