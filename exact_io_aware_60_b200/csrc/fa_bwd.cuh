@@ -296,8 +296,15 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int G = (int)gridDim.x;
         const int u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
         if (u >= p.num_tiles * p.BH) return false;
-        it.kt = u / p.BH;
-        it.bh = u - it.kt * p.BH;
+        if (D == 128) {
+            // head-major: the CTAs of a round share one or two heads, whose fp32 dQ
+            // accumulator then stays in L2 while every key tile reduces into it
+            it.bh = u / p.num_tiles;
+            it.kt = u - it.bh * p.num_tiles;
+        } else {
+            it.kt = u / p.BH;
+            it.bh = u - it.kt * p.BH;
+        }
         int L = p.N;
         if (p.kv_len != nullptr) {
             L = p.kv_len[it.bh / p.H];
