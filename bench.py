@@ -20,6 +20,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
+import re
 import json
 import math
 import os
@@ -129,12 +130,18 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the CUDA sources with comments removed and whitespace collapsed: a profile
+    summary stays valid across comment and layout edits and goes stale on any change to
+    the code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_60_b200", "csrc")
     for n in sorted(os.listdir(csrc)):
         if n.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(f.read())
+            with open(os.path.join(csrc, n), encoding="utf-8") as f:
+                src = f.read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
+            h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -240,10 +240,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Persistent CTA: work items are (key tile kt, head bh), numbered u = kt * BH + bh so
-    // that heavier causal tiles (small kt) come first.  Round r of CTA c takes item
-    // r * G + c on even rounds and r * G + (G - 1 - c) on odd ones (G = grid size); the
-    // zigzag evens out the causal work.  Every role walks the same list on its own.
+    // Persistent CTA: work items are (key tile kt, head bh), numbered u = kt * BH + bh at
+    // d = 64 so that heavier causal tiles (small kt) come first, and u = bh * T + kt at
+    // d = 128 (head-major: the long-sequence case, where one head's fp32 dQ accumulator
+    // should stay in L2).  Round r of CTA c takes item r * G + c on even rounds and
+    // r * G + (G - 1 - c) on odd ones (G = grid size); the zigzag evens out the causal
+    // work.  Every role walks the same list on its own.
 
     if (warp == C::W_TMA && lane == 0) {
         tma_prefetch_desc(&tmQ);
