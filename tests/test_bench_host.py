@@ -94,6 +94,22 @@ def test_profile_traffic_only_for_current_sources(tmp_path, monkeypatch):
     assert bench.profile_traffic("fa_bwd_kernel", "gpt2") is None
 
 
+def test_source_hash_ignores_comments_and_layout_only(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    csrc = tmp_path / "exact_io_aware_60_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    f = csrc / "k.cuh"
+    f.write_text("int a = 1;  // one\nint b = 2;\n")
+    h0 = bench.kernel_source_sha()
+    f.write_text("/* header\n   text */\nint a = 1;   // first value, reworded\n\n\nint b = 2;\n")
+    assert bench.kernel_source_sha() == h0
+    f.write_text("int a = 1;\nint b = 3;\n")
+    assert bench.kernel_source_sha() != h0
+    (csrc / "note.txt").write_text("not a CUDA source")
+    f.write_text("int a = 1;  // one\nint b = 2;\n")
+    assert bench.kernel_source_sha() == h0
+
+
 def test_visible_pairs_counts():
     import numpy as np
     T, N = 8, 1024
