@@ -129,19 +129,52 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_sha() -> str:
-    """Hash of the CUDA sources with comments removed and whitespace collapsed: a profile
+# The sources a kernel's profile depends on: its own header, the shared helpers, and the
+# host function in fa_api.cu that configures and launches it.
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": (("fa_fwd.cuh", "sm100.cuh", "dropout.cuh"), "launch_fwd"),
+    "fa_bwd_kernel": (("fa_bwd.cuh", "sm100.cuh", "dropout.cuh"), "launch_bwd"),
+}
+
+
+def _code_only(src: str) -> str:
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return " ".join(src.split())
+
+
+def _function_text(src: str, name: str) -> str:
+    """The text of the (non-template-specialised) host function ``int name(...) {...}``."""
+    start = src.find(f"int {name}(")
+    if start < 0:
+        return ""
+    end = src.find("\n}\n", start)
+    return src[start:end if end >= 0 else len(src)]
+
+
+def kernel_source_sha(kernel: str = None) -> str:
+    """Hash of CUDA code with comments removed and whitespace collapsed, so that a profile
     summary stays valid across comment and layout edits and goes stale on any change to
-    the code."""
+    the code.  With ``kernel`` (a key of KERNEL_SOURCES): only the files and the launch
+    function that kernel depends on; without: every source (for the launch list)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_60_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh")):
+    if kernel is None:
+        names = sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh")))
+        for n in names:
             with open(os.path.join(csrc, n), encoding="utf-8") as f:
-                src = f.read()
-            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            src = re.sub(r"//[^\n]*", "", src)
-            h.update(" ".join(src.split()).encode())
+                h.update(_code_only(f.read()).encode())
+        return h.hexdigest()[:16]
+    files, launcher = KERNEL_SOURCES[kernel]
+    for n in files:
+        path = os.path.join(csrc, n)
+        if os.path.exists(path):
+            with open(path, encoding="utf-8") as f:
+                h.update(_code_only(f.read()).encode())
+    api = os.path.join(csrc, "fa_api.cu")
+    if os.path.exists(api):
+        with open(api, encoding="utf-8") as f:
+            h.update(_code_only(_function_text(f.read(), launcher)).encode())
     return h.hexdigest()[:16]
 
 
@@ -159,7 +192,7 @@ def profile_traffic(kernel: str, workload: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("source_sha") != kernel_source_sha():
+    if vals.get("source_sha") != kernel_source_sha(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])

@@ -84,13 +84,24 @@ def test_profile_traffic_only_for_current_sources(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     csrc = tmp_path / "exact_io_aware_60_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cuh").write_text("kernel v1")
+    (csrc / "fa_bwd.cuh").write_text("kernel v1")
+    (csrc / "fa_fwd.cuh").write_text("forward v1")
+    (csrc / "fa_api.cu").write_text("int launch_bwd(int a) {\n  return a;\n}\nint launch_fwd(int b) {\n  return b;\n}\n")
     (tmp_path / "profiles").mkdir()
-    sha = bench.kernel_source_sha()
+    sha = bench.kernel_source_sha("fa_bwd_kernel")
     (tmp_path / "profiles" / "fa_bwd_kernel_gpt2.txt").write_text(
         f"source_sha: {sha}\ndram_bytes_per_launch: 12345\n")
     assert bench.profile_traffic("fa_bwd_kernel", "gpt2") == 12345.0
-    (csrc / "k.cuh").write_text("kernel v2")
+    # another kernel's code, or another launch function, does not touch this profile
+    (csrc / "fa_fwd.cuh").write_text("forward v2")
+    (csrc / "fa_api.cu").write_text("int launch_bwd(int a) {\n  return a;\n}\nint launch_fwd(int b) {\n  return b + 1;\n}\n")
+    assert bench.profile_traffic("fa_bwd_kernel", "gpt2") == 12345.0
+    # its own launch function or header does
+    (csrc / "fa_api.cu").write_text("int launch_bwd(int a) {\n  return a + 1;\n}\nint launch_fwd(int b) {\n  return b + 1;\n}\n")
+    assert bench.profile_traffic("fa_bwd_kernel", "gpt2") is None
+    (csrc / "fa_api.cu").write_text("int launch_bwd(int a) {\n  return a;\n}\nint launch_fwd(int b) {\n  return b + 1;\n}\n")
+    assert bench.profile_traffic("fa_bwd_kernel", "gpt2") == 12345.0
+    (csrc / "fa_bwd.cuh").write_text("kernel v2")
     assert bench.profile_traffic("fa_bwd_kernel", "gpt2") is None
 
 
