@@ -150,3 +150,16 @@ def test_dropout_and_block_sparse_are_exclusive():
         bench.main(["--impl", "reference", "--dropout", "0.1", "--block-sparse"])
     with pytest.raises(SystemExit):
         bench.main(["--impl", "reference", "--dropout", "1.0"])
+
+
+def test_profiled_kernels_have_their_sources_and_launchers():
+    """Every kernel whose profile bench.py reads names real files and a launch function
+    that exists in fa_api.cu (a rename must not silently drop it from the hash)."""
+    import os
+    csrc = os.path.join(bench.ROOT, "exact_io_aware_60_b200", "csrc")
+    api = open(os.path.join(csrc, "fa_api.cu"), encoding="utf-8").read()
+    for kernel, (files, launcher) in bench.KERNEL_SOURCES.items():
+        for n in files:
+            assert os.path.exists(os.path.join(csrc, n)), (kernel, n)
+        text = bench._function_text(api, launcher)
+        assert text.startswith(f"int {launcher}(") and "return FA_OK;" in text, kernel
