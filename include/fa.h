@@ -158,9 +158,10 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, void *stream);
 
 /*
- * Inference-shaped forward (aicassindra page, "Inference"; stackzen glossary, where the
- * savings of the method at inference are cited): Nq queries against Nk keys, Nq usually
- * much smaller than Nk (decoding, or a chunk of new tokens against a long cache).  The
+ * Inference-shaped forward (stackzen.ai glossary entry "FlashAttention", which cites the
+ * method's saving of memory traffic at inference as well as in training): Nq queries
+ * against Nk keys, Nq usually much smaller than Nk (decoding, or a chunk of new tokens
+ * against a long cache).  The
  * queries are the last Nq positions of the key sequence:
  *     key j is visible to query i  iff  j < kv_len[b]  and  (!causal or j <= i + Nk - Nq).
  * The key range is split into num_splits parts processed by separate CTAs (so that a
@@ -282,6 +283,10 @@ FA_API int fa_dropout_mask(int B, int H, int N, float p_drop, unsigned long long
  *
  * Set-up: the first call on each device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream capture begins.
+ * The cache is kept per device ordinal for the life of the process, so it assumes the
+ * device's primary context (the one the CUDA runtime uses) and no cudaDeviceReset in
+ * between: after a reset, or from another context on the same device, the cached
+ * address would be stale.
  *
  * Sharing: all calls share the one array, and it keeps the previous call's contents;
  * the call clears what must start at zero itself.  Two calls whose kernels may overlap

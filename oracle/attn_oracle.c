@@ -35,7 +35,7 @@
  * A row with no allowed key has O = 0, LSE = -inf, zero gradients.
  *
  * Queries and keys may differ in number (the inference shape: a short block of Nq new
- * queries against Nk cached keys, aicassindra page "Inference", stackzen glossary).  The
+ * queries against Nk cached keys; stackzen.ai glossary entry "FlashAttention").  The
  * queries are then the last Nq positions of the key sequence, so the causal rule reads
  *   allowed(i, j) = (j < L) && (!causal || j <= i + Nk - Nq),
  * which is the rule above when Nq = Nk.

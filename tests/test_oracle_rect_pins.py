@@ -1,6 +1,6 @@
 """Pins of the oracle for queries and keys of different lengths (the inference shape:
-a short block of new queries against a long key sequence, aicassindra page "Inference";
-stackzen glossary).  The Nq queries are the last Nq positions of the Nk-long sequence, so
+a short block of new queries against a long key sequence; stackzen.ai glossary entry
+"FlashAttention", which cites the method's saving at inference).  The Nq queries are the last Nq positions of the Nk-long sequence, so
 causal masking keeps key j for query i when j <= i + Nk - Nq.
 
 Fixed from outside the oracle by: brute-force softmax without the max shift on tiny
