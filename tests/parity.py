@@ -4,9 +4,17 @@ run the fp64 oracle on the same seeded inputs, and compare.
 Tolerances (fp16/bf16 inputs, fp32 accumulation): O max-abs <= 1e-2, LSE max-abs <= 1e-3,
 dQ/dK/dV relative L2 (||g - g_ref|| / ||g_ref|| over the whole tensor) <= 2e-2.
 
-O is returned in the 16-bit input dtype, whose spacing exceeds 2e-2 for |O| >= 4 (bf16),
-so the O bound is applied to the computation: element-wise |O - O_ref| <= 1e-2 plus half
-an ulp of O_ref in the output dtype.  The plain max-abs error is reported beside it.
+O is returned in the 16-bit input dtype.  Where |O_ref| >= 4 in bf16 the spacing is 2^-5,
+so rounding the exact value alone can be off by 2^-6 = 0.0156 > 1e-2 and no bf16 output
+can meet the bound there.  Element-wise, the graded rule is therefore
+    |O - O_ref| <= max(1e-2, halfulp(O_ref) + 2e-3),
+which is the plain 1e-2 bound wherever half an ulp plus the small computation allowance
+fits under it (|O| < 4 in bf16, every fp16 value below 8), and half an ulp plus 2e-3 only
+where it does not.  The plain max-abs error is reported beside the graded one.
+
+Gradients are also graded per (batch, head): a head's error norm over the larger of its
+own reference norm and the root-mean-square head norm stays <= 2e-2, so an error confined
+to part of one head cannot hide in the norm over all heads.
 """
 from __future__ import annotations
 
@@ -17,8 +25,12 @@ import oracle
 from exact_io_aware_60_b200 import fa
 
 O_ATOL = 1e-2
+# Allowance for the computation on top of half an ulp of output rounding, used only where
+# that sum exceeds O_ATOL (large |O|; see the module docstring).
+O_EPS = 2e-3
 LSE_ATOL = 1e-3
 GRAD_REL_L2 = 2e-2
+GRAD_REL_L2_HEAD = 2e-2
 
 # Fraction bits of the 16-bit output types.  O is returned in the input dtype, so on top of
 # the computation's error every output element carries up to half an ulp of rounding.
@@ -79,13 +91,15 @@ def half_ulp(x: np.ndarray, dtype) -> np.ndarray:
     return np.where(ax > 0, np.exp2(e - fb - 1), 0.0)
 
 
-def o_error_beyond_rounding(gpu_o: np.ndarray, ref_o: np.ndarray, dtype) -> float:
-    """max(|O_gpu - O_ref| - halfulp(O_ref)): the error of the computation once the
-    unavoidable rounding of the 16-bit output is set aside.  This is the graded O error:
-    it must stay <= O_ATOL.  (The plain max-abs is reported beside it.)"""
+def o_graded_error(gpu_o: np.ndarray, ref_o: np.ndarray, dtype) -> float:
+    """The graded O error, which must stay <= O_ATOL: max over elements of
+    |O_gpu - O_ref| - max(0, halfulp(O_ref) + O_EPS - O_ATOL).  An element passes exactly
+    when |O_gpu - O_ref| <= max(O_ATOL, halfulp(O_ref) + O_EPS); where half an ulp plus
+    O_EPS fits under O_ATOL the grade is the plain error."""
     if gpu_o.size == 0:
         return 0.0
-    return float(np.max(np.abs(gpu_o - ref_o) - half_ulp(ref_o, dtype)))
+    excess = np.maximum(0.0, half_ulp(ref_o, dtype) + O_EPS - O_ATOL)
+    return float(np.max(np.abs(gpu_o - ref_o) - excess))
 
 
 def rounding_floor(ref: np.ndarray, dtype) -> float:
@@ -106,7 +120,7 @@ def compare_forward(gpu: dict, ref: dict, mask=None) -> dict:
         go, gl, ro, rl = go[mask], gl[mask], ro[mask], rl[mask]
     o_err = float(np.max(np.abs(go - ro))) if go.size else 0.0
     ro_r = torch.from_numpy(np.ascontiguousarray(ro)).to(dtype).double().numpy()
-    res = {"o_err": o_error_beyond_rounding(go, ro, dtype), "o_max_abs": o_err,
+    res = {"o_err": o_graded_error(go, ro, dtype), "o_max_abs": o_err,
            "lse_max_abs": lse_err(gl, rl),
            "o_vs_rounded_oracle": float(np.max(np.abs(go - ro_r))) if go.size else 0.0,
            "o_rounding_floor": rounding_floor(ro, dtype)}
@@ -114,12 +128,34 @@ def compare_forward(gpu: dict, ref: dict, mask=None) -> dict:
     return res
 
 
+def head_rel_l2_max(g: np.ndarray, r: np.ndarray) -> float:
+    """Largest per-head error norm, each over max(that head's reference norm, the
+    root-mean-square head norm).  ``g``, ``r``: [heads, rows, d] (or [B, H, rows, d]).
+    The floor keeps heads whose exact gradient is zero (e.g. a sequence with one visible
+    key) from dividing rounding noise by zero."""
+    g = g.reshape(-1, *g.shape[-2:])
+    r = r.reshape(-1, *r.shape[-2:])
+    if g.shape[0] == 0:
+        return 0.0
+    num = np.sqrt(np.sum((g - r) ** 2, axis=(1, 2)))
+    den = np.sqrt(np.sum(r ** 2, axis=(1, 2)))
+    floor = np.sqrt(np.sum(den ** 2) / den.size)
+    if floor == 0.0:
+        return float(np.max(num))
+    return float(np.max(num / np.maximum(den, floor)))
+
+
 def compare_backward(gpu: dict, ref: dict, mask=None) -> dict:
+    """Relative L2 error of dQ, dK, dV over the selected heads (the graded figure,
+    <= GRAD_REL_L2) and the largest per-head figure (<= GRAD_REL_L2_HEAD, the same
+    bound).  Returns both kinds of keys; every value must stay within 2e-2."""
     res = {}
     for n in ("dq", "dk", "dv"):
         g, r = to_f64(gpu[n]), ref[n]
         if mask is not None:
             g, r = g[mask], r[mask]
         res[n + "_rel_l2"] = rel_l2(g, r)
+        res[n + "_head_max"] = head_rel_l2_max(g, r)
+    assert GRAD_REL_L2_HEAD == GRAD_REL_L2  # callers grade max(values) against one bound
     print("backward parity:", {k: f"{v:.3e}" for k, v in res.items()})
     return res

@@ -9,7 +9,7 @@ import oracle
 from exact_io_aware_60_b200 import fa
 from exact_io_aware_60_b200 import workloads as W
 from parity import (GRAD_REL_L2, LSE_ATOL, O_ATOL, compare_backward, compare_forward,
-                    o_error_beyond_rounding, oracle_full, rel_l2, rounding_floor, run_gpu,
+                    o_graded_error, oracle_full, rel_l2, rounding_floor, run_gpu,
                     to_f64)
 
 pytestmark = pytest.mark.gpu
@@ -122,7 +122,7 @@ def test_backward_causal64k_sampled():
         gdq = to_f64(gpu["dq"][b, h])[rows]
         go = to_f64(gpu["o"][b, h])[rows]
         errs = {"dq_rel_l2": rel_l2(gdq, ref["dq"]),
-                "o_err": o_error_beyond_rounding(go, ref["o"], w.dtype),
+                "o_err": o_graded_error(go, ref["o"], w.dtype),
                 "o_max_abs": float(np.max(np.abs(go - ref["o"]))),
                 "o_rounding_floor": rounding_floor(ref["o"], w.dtype)}
         # keys >= N - tail are seen only by rows >= N - tail, all of which are in `rows`

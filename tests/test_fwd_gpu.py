@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from exact_io_aware_60_b200 import workloads as W
-from parity import (LSE_ATOL, O_ATOL, compare_forward, o_error_beyond_rounding,
+from parity import (LSE_ATOL, O_ATOL, compare_forward, o_graded_error,
                     oracle_full, rounding_floor, run_gpu, to_f64)
 
 pytestmark = pytest.mark.gpu
@@ -88,7 +88,7 @@ def test_forward_long_workloads_sampled_rows(name, heads):
         go = to_f64(gpu["o"][b, h])[rows]
         gl = to_f64(gpu["lse"][b, h])[rows]
         o_max = float(np.max(np.abs(go - ref["o"])))
-        o_err = o_error_beyond_rounding(go, ref["o"], w.dtype)
+        o_err = o_graded_error(go, ref["o"], w.dtype)
         l_err = float(np.max(np.abs(gl - ref["lse"])))
         floor = rounding_floor(ref["o"], w.dtype)
         print(f"{name} head {(b, h)}: O error {o_err:.3e}, O max-abs {o_max:.3e} (output "

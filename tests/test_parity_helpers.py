@@ -2,7 +2,7 @@
 import numpy as np
 import torch
 
-from parity import half_ulp, o_error_beyond_rounding, rel_l2, rounding_floor
+from parity import O_ATOL, O_EPS, half_ulp, head_rel_l2_max, o_graded_error, rel_l2, rounding_floor
 
 
 def test_half_ulp_bounds_actual_rounding():
@@ -19,17 +19,54 @@ def test_half_ulp_bounds_actual_rounding():
         assert rounding_floor(x, dt) == np.max(err)
 
 
-def test_o_error_beyond_rounding():
-    ref = np.array([0.5, 5.0])
-    # an exactly rounded output has no error beyond rounding
-    out = torch.from_numpy(ref + 0.013).to(torch.bfloat16).double().numpy()
-    e = o_error_beyond_rounding(out, ref + 0.013, torch.bfloat16)
-    assert e <= 1e-12
-    # a computation error of 0.02 on top of rounding is visible
-    assert o_error_beyond_rounding(ref + 0.02, ref, torch.bfloat16) > 0.004
+def test_o_graded_error_is_plain_max_abs_below_4():
+    # Where half an ulp plus O_EPS fits under O_ATOL (|O| < 4 in bf16, < 8 in fp16) the
+    # grade is the plain absolute error: 0.0105 fails at every such magnitude, even where
+    # half an ulp alone is 0.0078 (bf16 in [2, 4)).
+    for dt, top in ((torch.bfloat16, 4.0), (torch.float16, 8.0)):
+        ref = np.array([0.01, 0.5, 1.5, 2.5, 3.9, top * 0.99])
+        for delta in (0.0042, -0.0099):
+            assert abs(o_graded_error(ref + delta, ref, dt) - abs(delta)) < 1e-15
+        assert o_graded_error(ref + 0.0105, ref, dt) > O_ATOL
+
+
+def test_o_graded_error_large_values():
+    # |O| in [4, 8) in bf16: spacing 2^-5, so exact rounding alone errs by up to 2^-6
+    ref = np.array([4.0 + 2.0 ** -6, 5.0 + 2.0 ** -6 - 1e-9, 7.5])
+    out = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+    assert np.max(np.abs(out - ref)) > O_ATOL              # the plain bound cannot hold
+    assert o_graded_error(out, ref, torch.bfloat16) <= O_ATOL   # the graded one does
+    # the allowance there is exactly half an ulp + O_EPS, and no more
+    ulp_half = 2.0 ** -6
+    assert o_graded_error(ref + ulp_half + O_EPS - 1e-6, ref, torch.bfloat16) <= O_ATOL
+    assert o_graded_error(ref + ulp_half + O_EPS + 1e-4, ref, torch.bfloat16) > O_ATOL
 
 
 def test_rel_l2():
     a = np.array([3.0, 4.0])
     assert rel_l2(a, a) == 0.0
     assert abs(rel_l2(a * 1.01, a) - 0.01) < 1e-12
+
+
+def test_head_rel_l2_max_finds_a_local_error():
+    rng = np.random.default_rng(1)
+    r = rng.standard_normal((4, 6, 256, 64))
+    g = r * (1 + 1e-3 * rng.standard_normal(r.shape))
+    assert head_rel_l2_max(g, r) < 2e-3
+    # a 32-row error of 10% in one head: invisible in the norm over all 24 heads at 2e-2,
+    # visible per head
+    bad = g.copy()
+    bad[2, 3, 100:132] *= 1.1
+    assert rel_l2(bad, r) < 2e-2
+    assert head_rel_l2_max(bad, r) > 2e-2
+
+
+def test_head_rel_l2_max_zero_reference_head():
+    # a head whose exact gradient is zero is measured against the RMS head norm
+    rng = np.random.default_rng(2)
+    r = rng.standard_normal((3, 128, 64))
+    r[1] = 0.0
+    g = r.copy()
+    g[1] = 1e-4
+    rms = np.sqrt(np.sum(r ** 2) / 3)
+    assert abs(head_rel_l2_max(g, r) - np.sqrt(128 * 64) * 1e-4 / rms) < 1e-12
