@@ -18,6 +18,7 @@ each step one bounded sample of the same workload; only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import re
@@ -132,8 +133,14 @@ def load_peaks():
 # The sources a kernel's profile depends on: its own header, the shared helpers, and the
 # host function in fa_api.cu that configures and launches it.
 KERNEL_SOURCES = {
-    "fa_fwd_kernel": (("fa_fwd.cuh", "sm100.cuh", "dropout.cuh"), "launch_fwd"),
-    "fa_bwd_kernel": (("fa_bwd.cuh", "sm100.cuh", "dropout.cuh"), "launch_bwd"),
+    "fa_fwd_kernel": (("fa_fwd.cuh", "sm100.cuh", "dropout.cuh"),
+                      ("launch_fwd", "make_map", "launch_pdl", "set_smem")),
+    "fa_bwd_kernel": (("fa_bwd.cuh", "sm100.cuh", "dropout.cuh"),
+                      ("launch_bwd", "bwd_workspace_layout", "make_map", "launch_pdl",
+                       "set_smem", "grid_for")),
+    "fa_bwd64_kernel": (("fa_bwd64.cuh", "fa_bwd.cuh", "sm100.cuh", "dropout.cuh"),
+                        ("launch_bwd", "bwd_workspace_layout", "make_map", "launch_pdl",
+                         "set_smem", "grid_for")),
 }
 
 
@@ -144,12 +151,19 @@ def _code_only(src: str) -> str:
 
 
 def _function_text(src: str, name: str) -> str:
-    """The text of the (non-template-specialised) host function ``int name(...) {...}``."""
-    start = src.find(f"int {name}(")
-    if start < 0:
-        return ""
-    end = src.find("\n}\n", start)
-    return src[start:end if end >= 0 else len(src)]
+    """The text of the top-level host function ``name`` in ``src``: from the line that
+    starts its definition (return type at the start of the line, the name followed by
+    ``(``, not a call or a declaration ending in ``;``) to its closing brace at the start
+    of a line.  Empty if there is no such definition."""
+    for m in re.finditer(rf"(?m)^[A-Za-z_][\w:<>, \t\*&]*\b{re.escape(name)}\(", src):
+        start = m.start()
+        brace = src.find("{", m.end())
+        semi = src.find(";", m.end())
+        if brace < 0 or (0 <= semi < brace):
+            continue  # a declaration
+        end = src.find("\n}\n", start)
+        return src[start:end + 3 if end >= 0 else len(src)]
+    return ""
 
 
 def kernel_source_sha(kernel: str = None) -> str:
@@ -165,7 +179,7 @@ def kernel_source_sha(kernel: str = None) -> str:
             with open(os.path.join(csrc, n), encoding="utf-8") as f:
                 h.update(_code_only(f.read()).encode())
         return h.hexdigest()[:16]
-    files, launcher = KERNEL_SOURCES[kernel]
+    files, functions = KERNEL_SOURCES[kernel]
     for n in files:
         path = os.path.join(csrc, n)
         if os.path.exists(path):
@@ -174,7 +188,9 @@ def kernel_source_sha(kernel: str = None) -> str:
     api = os.path.join(csrc, "fa_api.cu")
     if os.path.exists(api):
         with open(api, encoding="utf-8") as f:
-            h.update(_code_only(_function_text(f.read(), launcher)).encode())
+            src = f.read()
+        for fn in functions:
+            h.update(_code_only(_function_text(src, fn)).encode())
     return h.hexdigest()[:16]
 
 
@@ -399,6 +415,123 @@ def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0, fp8_set
                       + f" in {dt:.1f} s (nominal FLOPs)"}
 
 
+def bwd_kernel_name(w, args) -> str:
+    """The backward main kernel a measured path launches (the library's rule): the
+    four-issuer kernel at d = 64 without dropout when a key tile visits at least 16 query
+    tiles on average (half of them under causal masking), else the general kernel."""
+    tiles = (w.N + 127) // 128
+    mean_q_tiles = (tiles + 1) // 2 if w.causal else tiles
+    use64 = w.d == 64 and args.dropout == 0 and mean_q_tiles >= 16
+    return "fa_bwd64_kernel" if use64 else "fa_bwd_kernel"
+
+
+def config_dict(w, args, world: int) -> dict:
+    """The workload description both arms print (identical for the same flags)."""
+    mask = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
+    return {"workload": w.description
+            + (", E4M3 inputs (per-tensor scales), forward only" if args.fp8 else
+               ", inference forward (split-KV)" if w.inference else ", forward + backward")
+            + (", block-sparse local+global pattern" if args.block_sparse else "")
+            + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            **({"Nq": w.n_q} if w.inference else {}),
+            "flops_per_step": step_flops(w, mask, fwd_only=args.fp8)[2],
+            "parallelism": f"replicas x{world} (no collective)",
+            "l2": "inputs rotated over resident sets totalling more than twice the 126 MB L2, "
+                  "so each step reads data evicted from it"}
+
+
+def kernel_sample_pass(w, sets, nsets, stream, dev, steps):
+    """``steps`` steps with CUDA events recorded by the library around the forward kernel
+    and the backward main kernel (on the launch stream).  Returns {0: [(start, stop)],
+    1: [...]}; the caller reads the elapsed times."""
+    import torch
+    from exact_io_aware_60_b200 import fa
+    evs = {0: [], 1: []}
+    for which in (0, 1):
+        for _ in range(steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            b.record(stream)
+            evs[which].append((a, b))
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        fa.fa_set_timing_events(0, *evs[0][i])
+        fa.fa_set_timing_events(1, *evs[1][i])
+        run_step(w, sets[i % nsets])
+    fa.fa_set_timing_events(0)
+    fa.fa_set_timing_events(1)
+    torch.cuda.synchronize(dev)
+    return evs
+
+
+# Other workloads measured after the headline one (forward + backward each): the kernels'
+# TFLOP/s and fraction of the tensor peak, and for the key-padded BERT shape, which sits at
+# the ridge point, the forward's achieved HBM bandwidth and its effective FLOPs as well.
+OTHER_WORKLOADS = ("bert", "long16k", "causal64k")
+
+
+def fwd_compulsory_bytes(w) -> float:
+    """HBM bytes a forward pass must move: read Q, K, V, write O (16-bit) and LSE (fp32)."""
+    return float(w.B * w.H * w.N * (4 * w.d * 2 + 4))
+
+
+def effective_flops(w, kv_len) -> tuple:
+    """(forward, backward) FLOPs over the pairs the key-padding mask leaves visible (the
+    kernels skip padded key blocks): 4 d per visible (query, key) pair forward, 10 d
+    backward."""
+    if kv_len is None:
+        return w.nominal_flops()
+    L = [min(w.N, max(0, int(x))) for x in kv_len]
+    pairs = 0.0
+    for Lb in L:
+        pairs += sum(min(Lb, i + 1) for i in range(w.N)) if w.causal else float(w.N) * Lb
+    f = 4.0 * w.d * w.H * pairs
+    return f, 2.5 * f
+
+
+def measure_other_workload(name, dev, stream, steps, peak, hbm, args):
+    import torch
+    from exact_io_aware_60_b200 import workloads as W
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, seed=0)
+    first = alloc_set(w, inp, dev)
+    per_set = set_bytes(first)
+    nsets = 1 if per_set > 2 * 126 * 2 ** 20 else 2
+    sets = [first] + [alloc_set(w, W.make_inputs(w, seed=i), dev) for i in range(1, nsets)]
+    for i in range(3):
+        run_step(w, sets[i % nsets])
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        run_step(w, sets[i % nsets])
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    step_ms = a.elapsed_time(b) / steps
+    evs = kernel_sample_pass(w, sets, nsets, stream, dev, steps)
+    f_fwd, f_bwd = w.nominal_flops()
+    k_f = sum(x.elapsed_time(y) for x, y in evs[0]) / steps
+    k_b = sum(x.elapsed_time(y) for x, y in evs[1]) / steps
+    tf = lambda f, ms: f / (ms * 1e-3) / 1e12
+    fk, bk = "fa_fwd_kernel", bwd_kernel_name(w, args)
+    res = {"workload": w.description, "steps": steps, "inputs_sets": nsets,
+           "ms_per_step": step_ms, "tflops_step": tf(f_fwd + f_bwd, step_ms),
+           fk: {"ms": k_f, "tflops": tf(f_fwd, k_f), "frac": tf(f_fwd, k_f) / peak},
+           bk: {"ms": k_b, "tflops": tf(f_bwd, k_b), "frac": tf(f_bwd, k_b) / peak}}
+    if inp["kv_len"] is not None:
+        e_fwd, e_bwd = effective_flops(w, inp["kv_len"].tolist())
+        gbs = fwd_compulsory_bytes(w) / (k_f * 1e-3) / 1e9
+        res[fk].update({
+            "effective_tflops": tf(e_fwd, k_f), "effective_frac": tf(e_fwd, k_f) / peak,
+            "hbm_bytes": fwd_compulsory_bytes(w), "hbm_gbs": gbs, "hbm_frac": gbs / hbm})
+        res[bk].update({"effective_tflops": tf(e_bwd, k_b),
+                        "effective_frac": tf(e_bwd, k_b) / peak})
+    del sets, first
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -411,6 +544,9 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = W.WORKLOADS[args.workload]
+    if args.heads > 0:
+        w = dataclasses.replace(w, H=args.heads,
+                                description=w.description + f" (reduced to H={args.heads})")
     mask_np = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
     f_fwd, f_bwd, f_step = step_flops(w, mask_np, fwd_only=args.fp8)
 
@@ -442,19 +578,11 @@ def bench_ours(args, rank, world, local_rank):
     if status != fa.FA_OK:
         raise RuntimeError(f"device status {status} after warm-up")
 
-    # Per-kernel events (forward kernel, backward main kernel) around the launches of
-    # every `stride`-th step of the timed region (about 256 samples): an event between two
-    # kernels stops the next one from starting early, so most steps run without them.
+    # The headline region: K steps back to back, no per-kernel events (an event between two
+    # kernels keeps the next one from starting early under programmatic dependent launch).
     K = args.steps
-    stride = max(1, K // 256)
-    sampled = list(range(0, K, stride))
-    evs = {0: [], 1: []}
-    for which in (0, 1):
-        for _ in sampled:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            b.record(stream)
-            evs[which].append((a, b))
+    fa.fa_set_timing_events(0)
+    fa.fa_set_timing_events(1)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(gpu_pci_id(local_rank))
     clocks.start()
@@ -464,41 +592,36 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     clocks.mark("t0")
     start.record(stream)
-    si = 0
     for i in range(K):
-        if si < len(sampled) and sampled[si] == i:
-            fa.fa_set_timing_events(0, *evs[0][si])
-            fa.fa_set_timing_events(1, *evs[1][si])
-            si += 1
-        else:
-            fa.fa_set_timing_events(0)
-            fa.fa_set_timing_events(1)
         run_step(w, sets[i % nsets])
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks.mark("t1")
     barrier()
     torch.cuda.synchronize(dev)
-    fa.fa_set_timing_events(0)
-    fa.fa_set_timing_events(1)
     clk = clocks.stop()
     status = fa.fa_get_device_status()
     if status != fa.FA_OK:
         raise RuntimeError(f"device status {status} after the timed region")
     ms = start.elapsed_time(end)
     max_ms = max_over_ranks(ms, dev if world > 1 else None)
-    k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / len(evs[0])
-    fwd_only = w.inference or args.fp8
-    k_bwd = 0.0 if fwd_only else sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
     value = whole_job_tflops(f_step, world, K, max_ms)
+
+    # Per-kernel device times (forward kernel, backward main kernel) from a separate pass of
+    # the same steps on the same rotated inputs, with events around those two launches.
+    evs = kernel_sample_pass(w, sets, nsets, stream, dev, max(3, min(K, args.kernel_steps)))
+    fwd_only = w.inference or args.fp8
+    k_fwd = sum(a.elapsed_time(b) for a, b in evs[0]) / len(evs[0])
+    k_bwd = 0.0 if fwd_only else sum(a.elapsed_time(b) for a, b in evs[1]) / len(evs[1])
 
     def spread(pairs):
         ts = sorted(a.elapsed_time(b) for a, b in pairs)
         pick = lambda q: ts[min(len(ts) - 1, int(q * (len(ts) - 1) + 0.5))]
         return {"calls": len(ts), "median_ms": pick(0.5), "p10_ms": pick(0.1), "p90_ms": pick(0.9)}
-    per_call = {"fa_fwd_kernel": spread(evs[0])}
+    fwd_name, bwd_name = "fa_fwd_kernel", bwd_kernel_name(w, args)
+    per_call = {fwd_name: spread(evs[0])}
     if not fwd_only:
-        per_call["fa_bwd_kernel"] = spread(evs[1])
+        per_call[bwd_name] = spread(evs[1])
 
     # back-to-back steps on one input set (inputs warm in the 126 MB L2), labelled as such
     Kw = min(K, 200)
@@ -602,9 +725,9 @@ def bench_ours(args, rank, world, local_rank):
         peak *= 2.0  # E4M3 dense peak: the measured bf16 figure x the nominal ratio 4.5 / 2.25
     # the dominant kernel is the one with the larger device time per step
     if k_bwd >= k_fwd:
-        dom_name, dom_flops, dom_ms = "fa_bwd_kernel", f_bwd, k_bwd
+        dom_name, dom_flops, dom_ms = bwd_name, f_bwd, k_bwd
     else:
-        dom_name, dom_flops, dom_ms = "fa_fwd_kernel", f_fwd, k_fwd
+        dom_name, dom_flops, dom_ms = fwd_name, f_fwd, k_fwd
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
@@ -612,6 +735,8 @@ def bench_ours(args, rank, world, local_rank):
                                + (" x 2 (e4m3 / bf16 nominal)" if args.fp8 else ""),
                 "flops_per_launch": dom_flops, "launch_ms": dom_ms,
                 "launches_timed": len(evs[0]),
+                "timing": "CUDA events around each launch in a sampled pass after the "
+                          "headline region",
                 "traffic": profile_traffic(dom_name, w.name)}
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     if w.inference and f_fwd / inference_bytes(w) < peak * 1e3 / hbm:
@@ -626,6 +751,17 @@ def bench_ours(args, rank, world, local_rank):
         cpu = cpu_baseline_sample(w, inp, args.cpu_seconds, args.dropout,
                                   fp8_set=first if args.fp8 else None)
 
+    others = None
+    if (args.workload == DEFAULT_WORKLOAD and not (args.block_sparse or args.dropout or args.fp8)
+            and not args.no_other_workloads):
+        others = {}
+        for name in OTHER_WORKLOADS:
+            others[name] = measure_other_workload(name, dev, stream, args.other_steps, peak, hbm,
+                                                  args)
+        status = fa.fa_get_device_status()
+        if status != fa.FA_OK:
+            raise RuntimeError(f"device status {status} after the other workloads")
+
     per_rank_value = f_step * K / (ms * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -633,23 +769,20 @@ def bench_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if args.fp8 else {torch.bfloat16: "bf16", torch.float16: "f16"}[w.dtype],
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
-        "config": {"workload": w.description
-                   + (", E4M3 inputs (per-tensor scales), forward only" if args.fp8 else
-                      ", inference forward (split-KV)" if w.inference else ", forward + backward")
-                   + (", block-sparse local+global pattern" if args.block_sparse else "")
-                   + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
-                   "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                   **({"Nq": w.n_q} if w.inference else {}),
-                   "flops_per_step": f_step, "parallelism": f"replicas x{world} (no collective)",
-                   "l2": f"{nsets} resident input/output sets ({nsets * per_set / 2**20:.0f} MiB) "
-                         "rotated so each step reads data evicted from the 126 MB L2"},
+        "config": config_dict(w, args, world),
+        "l2_sets": f"{nsets} resident input/output sets ({nsets * per_set / 2**20:.0f} MiB)",
         "pct_of_peak": 100.0 * per_rank_value / peak,
-        "kernels": ({"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12}}
+        "kernels": ({fwd_name: {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12,
+                                "frac": f_fwd / (k_fwd * 1e-3) / 1e12 / peak}}
                     if fwd_only else
-                    {"fa_fwd_kernel": {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12},
-                     "fa_bwd_kernel": {"ms": k_bwd, "tflops": f_bwd / (k_bwd * 1e-3) / 1e12}}),
+                    {fwd_name: {"ms": k_fwd, "tflops": f_fwd / (k_fwd * 1e-3) / 1e12,
+                                "frac": f_fwd / (k_fwd * 1e-3) / 1e12 / peak},
+                     bwd_name: {"ms": k_bwd, "tflops": f_bwd / (k_bwd * 1e-3) / 1e12,
+                                       "frac": f_bwd / (k_bwd * 1e-3) / 1e12 / peak}}),
         "roofline": roofline,
         "per_call": per_call,
+        "kernel_times": "per-kernel figures from a separate pass of the same steps with "
+                        "events around the two kernels; the headline region has none",
         "warm_l2": warm,
         "peak_mem_bytes": peak_mem,
         "e2e": e2e,
@@ -658,6 +791,7 @@ def bench_ours(args, rank, world, local_rank):
                          else 4 * K),
         "clocks": clk,
         "cpu_baseline": cpu,
+        "other_workloads": others,
     }
     if world > 1:
         dist.barrier(device_ids=[local_rank])
@@ -733,14 +867,7 @@ def bench_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), GPT-2-small shapes; no dataset)",
-        "config": {"workload": w.description
-                   + (", E4M3 inputs (per-tensor scales), forward only" if args.fp8 else
-                      ", inference forward (split-KV)" if w.inference else ", forward + backward")
-                   + (", block-sparse local+global pattern" if args.block_sparse else "")
-                   + (f", dropout p={args.dropout}" if args.dropout > 0 else ""),
-                   "B": w.B, "H": w.H,
-                   "N": w.N, "d": w.d, "causal": w.causal,
-                   **({"Nq": w.n_q} if w.inference else {})},
+        "config": config_dict(w, args, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -759,6 +886,14 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-steps", type=int, default=64,
+                    help="steps of the per-kernel timing pass after the headline region")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the BERT / long16k / causal64k kernel measurements")
+    ap.add_argument("--other-steps", type=int, default=5)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling: run the workload with this many heads instead of its own "
+                         "(a smaller launch of the same kernel shape for counter captures)")
     ap.add_argument("--block-sparse", action="store_true",
                     help="measure the block-sparse path with a local+global block pattern "
                          "(FLOPs counted over the visible pairs only)")

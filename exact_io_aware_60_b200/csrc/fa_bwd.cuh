@@ -11,8 +11,10 @@
 // textbook derivatives of softmax and of the two products.)
 //
 // Three kernels, all on the caller's stream:
-//   1. fa_bwd_prep_kernel: D_i = rowsum(dO o O) in fp32, LSE in base 2 (padded to whole
-//      128-row tiles, +inf where there is no row), and zeroes the fp32 dQ accumulator.
+//   1. fa_bwd_prep_kernel: D_i = rowsum(dO o O) in fp32 and LSE in base 2, both stored
+//      negated (so that the main kernel's P = 2^(S scale log2e - LSE2) and dP - D are one
+//      packed fused multiply-add or add each), padded to whole 128-row tiles (-inf for the
+//      LSE where there is no row); and zeroes the fp32 dQ accumulator.
 //   2. fa_bwd_kernel: persistent CTAs (one per SM) walking (128-key tile, head) items, each
 //      looping over the 128-query tiles that can see its keys (causal: only tiles on or
 //      below the diagonal).
@@ -48,8 +50,8 @@ struct BwdPrepParams {
     const void *o;
     const void *dout;
     const float *lse;
-    float *lse2;   // [BH][Npad]
-    float *dvec;   // [BH][Npad]
+    float *nlse2;  // [BH][Npad]: -LSE in base 2 (-inf for padding rows)
+    float *ndvec;  // [BH][Npad]: -D (times dscale)
     float4 *dq_acc;
     long long dq_acc_vec4;  // number of float4 in dq_acc
     float dscale;           // D is stored times this (1, or 1 / keep_scale with dropout)
@@ -65,12 +67,16 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p) {
     constexpr int G = D / 8;           // threads per row
     constexpr int RPW = 32 / G;        // rows per warp step
-    pdl_wait();
-    pdl_launch_dependents();
     const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long nthreads = (long long)gridDim.x * blockDim.x;
+    // The accumulator is the backward pass's own scratch, which no earlier kernel of the
+    // stream reads or writes while this call runs: it is zeroed before the wait, so that
+    // the zeroing overlaps the tail of the kernel before (the forward pass, in a training
+    // step).  O and dO may be that kernel's outputs, so they are read after the wait.
     for (long long i = tid; i < p.dq_acc_vec4; i += nthreads)
         p.dq_acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    pdl_wait();
+    pdl_launch_dependents();
     const long long rows_total = p.BH * p.Npad;
     const int lane = threadIdx.x & 31;
     const int g = lane % G;
@@ -79,7 +85,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
     for (long long base = warp_id * RPW; base < rows_total; base += nwarps * RPW) {
         const long long rr = base + lane / G;
         float acc = 0.f;
-        float l2 = INFINITY;
+        float l2 = INFINITY;  // LSE in base 2; +inf (P = 0) for rows that do not exist
         if (rr < rows_total) {
             const long long bh = rr / p.Npad;
             const int r = (int)(rr - bh * p.Npad);
@@ -105,8 +111,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
 #pragma unroll
         for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (g == 0 && rr < rows_total) {
-            p.dvec[rr] = acc * p.dscale;
-            p.lse2[rr] = l2;
+            p.ndvec[rr] = -acc * p.dscale;
+            p.nlse2[rr] = -l2;
         }
     }
 }
@@ -117,24 +123,28 @@ template <bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_convert_kernel(const float4 *acc, uint2 *out,
                                                              long long n_vec4, float scale) {
     pdl_wait();
-    pdl_launch_dependents();
     const long long nthreads = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec4; i += nthreads) {
         const float4 a = acc[i];
         out[i] = make_uint2(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale));
     }
+    // Only now may the next kernel start: the next backward call's preprocess zeroes this
+    // accumulator before it waits (the same workspace, or the static one, may be reused).
+    pdl_launch_dependents();
 }
 
 // --------------------------------------------------------------------------- main
 
 struct BwdParams {
-    const float *lse2;  // [BH][Npad], log2-domain LSE (+inf for padding rows)
+    const float *nlse2;  // [BH][Npad], minus the log2-domain LSE (-inf for padding rows)
     // Block-sparse attention: uint8 [heads][T][T]; key tile kt visits only the query tiles
     // qi with mask[qi][kt] != 0.  nullptr = dense.
     const uint8_t *bmask;
     long long bmask_bh_stride;  // 0: one mask for every (batch, head)
-    const float *dvec;  // [BH][Npad]
+    const float *ndvec;  // [BH][Npad], -D
     float *dq_acc;      // [BH][N][D] fp32
+    void *dk;           // [BH][N][D] 16-bit outputs (written from registers by the d = 64
+    void *dv;           // kernel; the general kernel stores them through TMA maps)
     const int *kv_len;
     int N;
     int Npad;
@@ -204,6 +214,7 @@ struct BwdBars {
     uint64_t do_full[3];
     uint64_t stage_empty[3];
     uint64_t dq_stage_free;  // d = 128: the dQ drain has finished with the dS buffer
+    uint64_t dp_read;  // d = 64: every P/dS warp has read dP^T (its columns may take the next)
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
         dkv_full, dkv_empty;
     uint32_t tmem_base;
@@ -267,6 +278,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bars->p_full, 256);
         mbar_init(&bars->p_free, 1);
         mbar_init(&bars->ds_full, 256);
+        mbar_init(&bars->dp_read, 256);
         mbar_init(&bars->ds_empty, 1);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 128);
@@ -334,12 +346,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int hf = 0; hf < C::HALVES; ++hf)
                     tma_load_3d(sQ + s * C::TILE + hf * C::HALF, &tmQ, &bars->q_full[s], hf * 64,
                                 qi * 128, bh);
-                bulk_load(sLSE + s * 128, p.lse2 + vec_off, 512, &bars->q_full[s]);
+                bulk_load(sLSE + s * 128, p.nlse2 + vec_off, 512, &bars->q_full[s]);
                 mbar_arrive_expect_tx(&bars->do_full[s], C::TILE + 512);
                 for (int hf = 0; hf < C::HALVES; ++hf)
                     tma_load_3d(sdO + s * C::TILE + hf * C::HALF, &tmdO, &bars->do_full[s],
                                 hf * 64, qi * 128, bh);
-                bulk_load(sDv + s * 128, p.dvec + vec_off, 512, &bars->do_full[s]);
+                bulk_load(sDv + s * 128, p.ndvec + vec_off, 512, &bars->do_full[s]);
                 return true;
             };
             bool ok = true;
@@ -417,13 +429,30 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if (C::P_OWN && gi > 0 && !mbar_wait(&bars->s_free, (gi - 1) & 1)) break;
                     if (!mbar_wait(&bars->q_full[s0], (gi / C::QS) & 1)) break;
                     tc_fence_after();
-                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s0));
-                    mma_commit(&bars->s_full);
-                    if (D == 128 && gi > 0 && !mbar_wait(&bars->dq_empty, (gi - 1) & 1)) break;
-                    if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
-                    tc_fence_after();
-                    mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s0));
-                    mma_commit(&bars->dp_full);
+                    if (D == 64) {
+                        // S^T and dP^T as two interleaved chains (MMAs into one accumulator
+                        // run one after the other; independent ones overlap)
+                        if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
+                            mma_ss(tmem + C::COL_S, k_kmaj + off, q_kmaj + stage_off(s0) + off, kIdescSq,
+                                   kk > 0 ? 1u : 0u);
+                            mma_ss(tmem + C::COL_DP, v_kmaj + off, do_kmaj + stage_off(s0) + off, kIdescSq,
+                                   kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&bars->s_full);
+                        mma_commit(&bars->dp_full);
+                    } else {
+                        mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s0));
+                        mma_commit(&bars->s_full);
+                        if (gi > 0 && !mbar_wait(&bars->dq_empty, (gi - 1) & 1)) break;
+                        if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s0));
+                        mma_commit(&bars->dp_full);
+                    }
                 }
                 for (int i = 0; i < n; ++i) {
                     const int g = gi + i;  // global iteration: ring stage and barrier phases
@@ -445,6 +474,15 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE,
                                do_mn + stage_off(s), i > 0);
                     mma_commit(&bars->p_free);
+                    if (D == 64 && i + 1 < n) {
+                        // dS^T_i goes to the P^T columns, so dP^T_{i+1} may overwrite dP^T_i
+                        // as soon as every P/dS warp has read it, ahead of dK_i and dQ_i.
+                        if (!mbar_wait(&bars->dp_read, g & 1) ||
+                            !mbar_wait(&bars->do_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
+                        mma_commit(&bars->dp_full);
+                    }
                     if (!C::P_OWN && i + 1 < n) {
                         // P^T_i lives in the S^T columns: S_{i+1} follows dV_i.
                         if (!mbar_wait(&bars->q_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
@@ -454,24 +492,34 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                     if (!mbar_wait(&bars->ds_full, g & 1)) { ok = false; break; }
                     tc_fence_after();
-                    mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
-                               q_mn + stage_off(s), i > 0);
-                    if (D == 64 && g > 0) {
-                        if (!mbar_wait(&bars->dq_empty, (g - 1) & 1)) { ok = false; break; }
+                    if (D == 64) {
+                        // dK_i and dQ_i as two interleaved chains (dQ has columns of its own)
+                        if (g > 0 && !mbar_wait(&bars->dq_empty, (g - 1) & 1)) { ok = false; break; }
                         tc_fence_after();
-                    }
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
-                               k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            mma_ts(tmem + C::COL_DK,  // dS^T_i from the P^T columns
+                                   tmem + C::COL_P + (kk >> 2) * C::P_HALF_STRIDE + (kk & 3) * 8,
+                                   q_mn + stage_off(s) + (uint64_t)(kk * 2048 >> 4), kIdescTs,
+                                   (i > 0 || kk > 0) ? 1u : 0u);
+                            mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
+                                   k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
+                        }
+                    } else {
+                        // dQ is written over dS^T, which dK reads: dK first
+                        mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
+                                   q_mn + stage_off(s), i > 0);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
+                                   k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
+                    }
                     mma_commit(&bars->dq_full);
                     mma_commit(&bars->ds_empty);
                     mma_commit(&bars->stage_empty[s]);
-                    if (i + 1 < n) {
-                        if (D == 128) {
-                            // dQ_i lives in the dP^T columns: wait until it has been drained.
-                            if (!mbar_wait(&bars->dq_empty, g & 1)) { ok = false; break; }
-                        }
+                    if (D == 128 && i + 1 < n) {
+                        // dQ_i lives in the dP^T columns: wait until it has been drained.
+                        if (!mbar_wait(&bars->dq_empty, g & 1)) { ok = false; break; }
                         if (!mbar_wait(&bars->do_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
                         tc_fence_after();
                         mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
@@ -495,7 +543,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int rr = 0; ok && item_at(rr, it); ++rr) {
         const int bh = it.bh;
         for (int i = 0, qi = it.q_first; i < it.n; ++i, qi = next_q(it, qi + 1)) {
-            if (!mbar_wait(&bars->dq_full, (gi + i) & 1)) { ok = false; break; }
+            // The 128 drain threads agree on the wait's outcome before the warp-wide TMEM
+            // loads and the named barriers below, so a timeout makes all of them leave.
+            if (!named_bar_and(2, 128, mbar_wait(&bars->dq_full, (gi + i) & 1))) { ok = false; break; }
             tc_fence_after();
             // Boxes of [128 rows][32 fp32], 16-byte chunks swizzled by row % 8, staged
             // ROUND_BOXES at a time (all D/32 at d = 64; two per round in the dS buffer at
@@ -572,7 +622,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     kb[u] = transpose16x16_halfwarp(a | (c << 16), lane);
                 }
             }
-            if (!mbar_wait(&bars->s_full, g & 1) || !mbar_wait(&bars->q_full[s], (g / C::QS) & 1)) {
+            // (waits are voted on per warp: the loop body has warp-wide TMEM loads and stores)
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, g & 1) &&
+                                             mbar_wait(&bars->q_full[s], (g / C::QS) & 1))) {
                 ok = false;
                 break;
             }
@@ -587,30 +639,34 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tc_fence_before();
                     mbar_arrive(&bars->s_free);  // S^T may now be overwritten by S_{i+1}
                 }
-                const float *lse2 = sLSE + s * 128 + h * 64;
+                const float *nl2 = sLSE + s * 128 + h * 64;  // -LSE2 of the 64 queries
+                const float2 sl2x2 = make_float2(sl2, sl2);
                 // Masks only on the causal diagonal tile and the key-padding tail tile.
                 const bool diag = p.causal && (qi == kt);
                 const bool tile_masked = diag || (kt * 128 + 128 > L);
                 if (!tile_masked) {
+                    // the exponent argument as one packed fused multiply-add per pair
 #pragma unroll
                     for (int k = 0; k < 64; k += 4) {
-                        const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + k);
-                        const float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
-                        const float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
-                        const float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
-                        const float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
-                        Pw[k >> 1] = pack2<BF16>(p0, p1);
-                        Pw[(k >> 1) + 1] = pack2<BF16>(p2, p3);
+                        const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k);
+                        const float2 x01 = __ffma2_rn(
+                            make_float2(__uint_as_float(w[k]), __uint_as_float(w[k + 1])), sl2x2,
+                            make_float2(l4.x, l4.y));
+                        const float2 x23 = __ffma2_rn(
+                            make_float2(__uint_as_float(w[k + 2]), __uint_as_float(w[k + 3])), sl2x2,
+                            make_float2(l4.z, l4.w));
+                        Pw[k >> 1] = pack2<BF16>(ex2(x01.x), ex2(x01.y));
+                        Pw[(k >> 1) + 1] = pack2<BF16>(ex2(x23.x), ex2(x23.y));
                     }
                 } else {
 #pragma unroll
                     for (int k = 0; k < 64; k += 4) {
                         const int c = h * 64 + k;  // query column in the tile
-                        const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + k);
-                        float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, -l4.x));
-                        float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, -l4.y));
-                        float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, -l4.z));
-                        float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, -l4.w));
+                        const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k);
+                        float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, l4.x));
+                        float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, l4.y));
+                        float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, l4.z));
+                        float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, l4.w));
                         // keys past the valid length, and queries before the key (causal)
                         if (!key_ok || (diag && c < t)) p0 = 0.f;
                         if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
@@ -621,7 +677,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                 }
             }
-            if (C::P_OWN && g > 0 && !mbar_wait(&bars->p_free, (g - 1) & 1)) {  // dV_{g-1} read P
+            // d = 64: the P^T columns last held dS^T_{g-1}: dK_{g-1} (issued after dV_{g-1})
+            // must have read it
+            if (C::P_OWN && g > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait(&bars->ds_empty, (g - 1) & 1))) {
                 ok = false;
                 break;
             }
@@ -640,38 +699,55 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(&bars->p_full);
 
-            if (!mbar_wait(&bars->dp_full, g & 1) || !mbar_wait(&bars->do_full[s], (g / C::QS) & 1) ||
-                (g > 0 && !mbar_wait(&bars->ds_empty, (g - 1) & 1)) ||
-                // d = 128: the dQ drain has staged dQ_{g-1} through the dS buffer and let go
-                (C::DQ_IN_DS && g > 0 && !mbar_wait(&bars->dq_stage_free, (g - 1) & 1))) {
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&bars->dp_full, g & 1) &&
+                                mbar_wait(&bars->do_full[s], (g / C::QS) & 1) &&
+                                (g == 0 || mbar_wait(&bars->ds_empty, (g - 1) & 1)) &&
+                                // d = 128: the dQ drain has staged dQ_{g-1} through the dS
+                                // buffer and let go
+                                (!C::DQ_IN_DS || g == 0 ||
+                                 mbar_wait(&bars->dq_stage_free, (g - 1) & 1)))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const float *dv = sDv + s * 128 + h * 64;
+            const float *ndv = sDv + s * 128 + h * 64;  // -D of the 64 queries
             uint32_t wdp[64];
             tmem_ld64(tmem + lane_base + C::COL_DP + h * 64, wdp);
+            if (C::P_OWN) {
+                tc_fence_before();
+                mbar_arrive(&bars->dp_read);  // dP^T may now be overwritten by dP^T_{g+1}
+                // dS^T goes over P^T, which dV_g must have read
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->p_free, g & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const uint32_t *w = wdp + cc * 32;
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const float2 d2 = *reinterpret_cast<const float2 *>(dv + cc * 32 + k);
+                    const float2 nd2 = *reinterpret_cast<const float2 *>(ndv + cc * 32 + k);
                     float dp0 = __uint_as_float(w[k]);
                     float dp1 = __uint_as_float(w[k + 1]);
                     if constexpr (DROP) {
                         if (!((kb[cc] >> (k >> 1)) & 1u)) dp0 = 0.f;
                         if (!((kb[cc] >> ((k >> 1) + 16)) & 1u)) dp1 = 0.f;
                     }
-                    // dS = P o (dP - D): the difference in fp32, rounded to 16 bits, times
-                    // the 16-bit P pair in one packed multiply
-                    pk[k >> 1] = mul2<BF16>(Pw[cc * 16 + (k >> 1)],
-                                            pack2<BF16>(dp0 - d2.x, dp1 - d2.y));
+                    // dS = P o (dP - D): the difference in fp32 (one packed add), rounded to
+                    // 16 bits, times the 16-bit P pair in one packed multiply
+                    const float2 diff = __fadd2_rn(make_float2(dp0, dp1), nd2);
+                    pk[k >> 1] = mul2<BF16>(Pw[cc * 16 + (k >> 1)], pack2<BF16>(diff.x, diff.y));
                 }
-                // dS^T pairs -> TMEM, over dP^T columns this warp has just read; A operand
-                // of dK += dS^T Q.
-                tmem_st16(tmem + lane_base + C::COL_DP + h * C::DS_HALF_STRIDE + cc * 16, pk);
+                // dS^T pairs -> TMEM, the A operand of dK += dS^T Q: over P^T_g at d = 64,
+                // over the dP^T columns this warp has just read at d = 128.
+                if (C::P_OWN)
+                    tmem_st16(tmem + lane_base + C::COL_P + h * C::P_HALF_STRIDE + cc * 16, pk);
+                else
+                    tmem_st16(tmem + lane_base + C::COL_DP + h * C::DS_HALF_STRIDE + cc * 16, pk);
                 // dS -> shared memory as the MN-major A operand of dQ = dS K:
                 // [query block h (64 queries)][key row t][128 bytes], 128-byte swizzle.
                 uint8_t *rowp = sdS + h * 16384 + t * 128;
@@ -698,6 +774,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                  (!C::DQ_IN_DS || mbar_wait(&bars->dq_stage_free, (gi + n - 1) & 1));
             tc_fence_after();
         }
+        // Agree again, so that the `break` after the epilogue is taken by all 256 threads
+        // or by none (the next item's epilogue barriers need every one of them).
+        ok = named_bar_and(1, 256, ok);
         // Staging in the dS buffer (free: every MMA of the item is done; 32 KB): both
         // 16-bit tiles at d = 64, one tile per round at d = 128.  Each warp converts its
         // lane quarter's D/2 columns.

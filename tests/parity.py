@@ -91,15 +91,21 @@ def half_ulp(x: np.ndarray, dtype) -> np.ndarray:
     return np.where(ax > 0, np.exp2(e - fb - 1), 0.0)
 
 
-def o_graded_error(gpu_o: np.ndarray, ref_o: np.ndarray, dtype) -> float:
+def o_graded_error(gpu_o: np.ndarray, ref_o: np.ndarray, dtype, out_scale: float = 1.0) -> float:
     """The graded O error, which must stay <= O_ATOL: max over elements of
     |O_gpu - O_ref| - max(0, halfulp(O_ref) + O_EPS - O_ATOL).  An element passes exactly
     when |O_gpu - O_ref| <= max(O_ATOL, halfulp(O_ref) + O_EPS); where half an ulp plus
-    O_EPS fits under O_ATOL the grade is the plain error."""
+    O_EPS fits under O_ATOL the grade is the plain error.
+
+    ``out_scale`` s > 1 is for outputs that are s times a convex combination of rows of V
+    (attention dropout, s = 1 / (1 - p)): their computation error scales with s, so the
+    bounds apply to O / s, i.e. |O_gpu - O_ref| <= max(s O_ATOL, halfulp(O_ref) + s O_EPS),
+    reported in units of O / s."""
     if gpu_o.size == 0:
         return 0.0
-    excess = np.maximum(0.0, half_ulp(ref_o, dtype) + O_EPS - O_ATOL)
-    return float(np.max(np.abs(gpu_o - ref_o) - excess))
+    s = float(out_scale)
+    excess = np.maximum(0.0, half_ulp(ref_o, dtype) + s * O_EPS - s * O_ATOL)
+    return float(np.max(np.abs(gpu_o - ref_o) - excess)) / s
 
 
 def rounding_floor(ref: np.ndarray, dtype) -> float:
@@ -109,7 +115,7 @@ def rounding_floor(ref: np.ndarray, dtype) -> float:
     return float(np.max(np.abs(r - ref))) if ref.size else 0.0
 
 
-def compare_forward(gpu: dict, ref: dict, mask=None) -> dict:
+def compare_forward(gpu: dict, ref: dict, mask=None, out_scale: float = 1.0) -> dict:
     """Max-abs errors of O and LSE over the entries selected by ``mask`` (a boolean
     [B,H] array of checked heads; None = all).  Also reports the error of O against the
     oracle rounded to the output dtype and the rounding floor itself (diagnostics)."""
@@ -120,7 +126,7 @@ def compare_forward(gpu: dict, ref: dict, mask=None) -> dict:
         go, gl, ro, rl = go[mask], gl[mask], ro[mask], rl[mask]
     o_err = float(np.max(np.abs(go - ro))) if go.size else 0.0
     ro_r = torch.from_numpy(np.ascontiguousarray(ro)).to(dtype).double().numpy()
-    res = {"o_err": o_graded_error(go, ro, dtype), "o_max_abs": o_err,
+    res = {"o_err": o_graded_error(go, ro, dtype, out_scale), "o_max_abs": o_err,
            "lse_max_abs": lse_err(gl, rl),
            "o_vs_rounded_oracle": float(np.max(np.abs(go - ro_r))) if go.size else 0.0,
            "o_rounding_floor": rounding_floor(ro, dtype)}

@@ -158,8 +158,50 @@ def test_profiled_kernels_have_their_sources_and_launchers():
     import os
     csrc = os.path.join(bench.ROOT, "exact_io_aware_60_b200", "csrc")
     api = open(os.path.join(csrc, "fa_api.cu"), encoding="utf-8").read()
-    for kernel, (files, launcher) in bench.KERNEL_SOURCES.items():
+    for kernel, (files, functions) in bench.KERNEL_SOURCES.items():
         for n in files:
             assert os.path.exists(os.path.join(csrc, n)), (kernel, n)
+        launcher = functions[0]
         text = bench._function_text(api, launcher)
         assert text.startswith(f"int {launcher}(") and "return FA_OK;" in text, kernel
+        # the helpers the launcher calls (tensor maps, workspace layout, launch) are hashed
+        # too, and each must be found as a definition
+        for fn in functions[1:]:
+            t = bench._function_text(api, fn)
+            assert t and f"{fn}(" in t.splitlines()[0] and t.rstrip().endswith("}"), (kernel, fn)
+            assert fn in text, (kernel, fn, "not called by the launcher")
+
+
+def test_function_text_skips_declarations_and_calls():
+    src = ("int helper(int a);\n"
+           "static int user(int b) {\n    return helper(b) + 1;\n}\n"
+           "int helper(int a) {\n    return a * 2;\n}\n")
+    t = bench._function_text(src, "helper")
+    assert t.startswith("int helper(int a) {") and "a * 2" in t
+    assert bench._function_text(src, "missing") == ""
+
+
+def test_reference_arm_config_matches_ours():
+    """Both arms print the same config dict for the same flags (so the two lines are
+    recognisably the same workload)."""
+    import argparse
+    from exact_io_aware_60_b200 import workloads as W
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3",
+                           "--workload", "tiny"]) == 0
+    d = json.loads(buf.getvalue().strip().splitlines()[-1])
+    args = argparse.Namespace(block_sparse=False, fp8=False, dropout=0.0)
+    assert d["config"] == bench.config_dict(W.WORKLOADS["tiny"], args, 1)
+    for key in ("flops_per_step", "parallelism", "l2", "workload"):
+        assert key in d["config"]
+
+
+def test_effective_flops_of_key_padding():
+    from exact_io_aware_60_b200 import workloads as W
+    w = W.WORKLOADS["bert"]
+    assert bench.effective_flops(w, [w.N] * w.B) == w.nominal_flops()
+    f, b = bench.effective_flops(w, [w.N // 2] * w.B)
+    assert f == w.nominal_flops()[0] / 2 and b == 2.5 * f
+    g = W.WORKLOADS["gpt2"]
+    assert bench.effective_flops(g, [g.N] * g.B)[0] == 4.0 * g.d * g.B * g.H * g.N * (g.N + 1) / 2

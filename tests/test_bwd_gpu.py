@@ -47,6 +47,33 @@ def test_backward_edge_shapes(N, d, dtype, causal, kvr):
             assert torch.all(gpu["dk"][b, :, L:] == 0) and torch.all(gpu["dv"][b, :, L:] == 0)
 
 
+# d = 64 from 4096 rows up runs the four-issuer backward kernel: ragged tails, causal
+# masking, key padding (including an empty sequence) at that size.
+LONG_EDGE = [
+    # (N, dtype, causal, kv_len_range)
+    (4096, torch.bfloat16, True, None),
+    (4173, torch.float16, False, None),
+    (4224, torch.bfloat16, True, (0, 4224)),
+    (4353, torch.bfloat16, False, (1, 4353)),
+]
+
+
+@pytest.mark.parametrize("N,dtype,causal,kvr", LONG_EDGE)
+def test_backward_long_d64_edge_shapes(N, dtype, causal, kvr):
+    w = W.custom(B=2, H=1, N=N, d=64, dtype=dtype, causal=causal, kv_len_range=kvr)
+    inp = W.make_inputs(w, seed=2000 + N)
+    gpu = run_gpu(inp, w.scale, causal)
+    ref = oracle_full(inp, w.scale, causal)
+    f = compare_forward(gpu, ref)
+    g = compare_backward(gpu, ref)
+    assert f["o_err"] <= O_ATOL and f["lse_max_abs"] <= LSE_ATOL, f
+    assert max(g.values()) <= GRAD_REL_L2, g
+    if kvr is not None:
+        for b in range(w.B):
+            L = int(inp["kv_len"][b])
+            assert torch.all(gpu["dk"][b, :, L:] == 0) and torch.all(gpu["dv"][b, :, L:] == 0)
+
+
 def test_backward_zero_length_sequence():
     w = W.custom(B=2, H=2, N=160, d=64, dtype=torch.bfloat16)
     inp = W.make_inputs(w, seed=11)

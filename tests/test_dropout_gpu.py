@@ -4,7 +4,9 @@ against the fp64 oracle with the same (p, seed, offset).
 The mask is integer work, so it is compared exactly: through fa_dropout_mask, and inside
 the fused kernels by inputs that make every mask bit visible in the outputs (Q = 0 gives
 uniform probabilities; one-hot rows of V, or of dO, then read the kept keys out of O, or
-the kept queries out of dV).  The floating-point results use the dense tolerances."""
+the kept queries out of dV).  The floating-point results use the dense tolerances, with O
+graded as O / r (r = 1 / (1 - p), the factor that scales every kept weight, and with it
+every rounding error of the weights), plus half an ulp of the output itself."""
 import numpy as np
 import pytest
 import torch
@@ -37,6 +39,11 @@ def test_mask_bit_exact(B, H, N, p, seed, offset):
     torch.cuda.synchronize()
     ref = oracle_mask(B, H, N, p, seed, offset)
     assert np.array_equal(keep.cpu().numpy(), ref)
+
+
+def keep_scale(p):
+    """The library's r = 256 / (256 - t), t = rint(256 p): the multiplier of kept weights."""
+    return 256.0 / (256 - int(np.rint(256 * p)))
 
 
 def run_dropout(q, k, v, do, *, scale, causal, kv_len, p, seed, offset, backward=True):
@@ -135,7 +142,7 @@ def test_dropout_matches_oracle(B, H, N, d, dtype, causal, kvr, p, seed):
     kv = None if inp["kv_len"] is None else inp["kv_len"].numpy()
     ref = oracle.attention(*(to_f64(inp[n]) for n in ("q", "k", "v", "do")), scale=w.scale,
                            causal=causal, kv_len=kv, dropout_p=p, seed=seed, offset=off)
-    f = compare_forward(gpu, ref)
+    f = compare_forward(gpu, ref, out_scale=keep_scale(p))
     g = compare_backward(gpu, ref)
     assert f["o_err"] <= O_ATOL and f["lse_max_abs"] <= LSE_ATOL, f
     assert max(g.values()) <= GRAD_REL_L2, g
@@ -148,7 +155,11 @@ def test_zero_probability_matches_dense_path():
                        kv_len=None, p=0.0, seed=1, offset=0)
     from parity import run_gpu
     dense = run_gpu(inp, w.scale, True)
-    assert torch.equal(drop["lse"], dense["lse"])
+    # at d = 64 the dense path has its own kernel (split rows, 3/8 of the exponentials from
+    # a polynomial with relative error <= 7.5e-5): the same LSE up to that error in the
+    # normaliser and fp32 summation order
+    assert torch.allclose(drop["lse"], dense["lse"], atol=2e-4, rtol=0), \
+        (drop["lse"] - dense["lse"]).abs().max()
     for n in ("o", "dq", "dk", "dv"):
         a, b = drop[n].float(), dense[n].float()
         assert torch.allclose(a, b, atol=2e-2, rtol=2e-2), (n, (a - b).abs().max())
@@ -180,7 +191,7 @@ def test_gpt2_shape_sampled_rows():
     mask = np.zeros((w.B, w.H), bool)
     for b, h in heads:
         mask[b, h] = True
-    f = compare_forward(gpu, ref, mask)
+    f = compare_forward(gpu, ref, mask, out_scale=keep_scale(p))
     g = compare_backward(gpu, ref, mask)
     assert f["o_err"] <= O_ATOL and f["lse_max_abs"] <= LSE_ATOL, f
     assert max(g.values()) <= GRAD_REL_L2, g

@@ -70,3 +70,14 @@ def test_head_rel_l2_max_zero_reference_head():
     g[1] = 1e-4
     rms = np.sqrt(np.sum(r ** 2) / 3)
     assert abs(head_rel_l2_max(g, r) - np.sqrt(128 * 64) * 1e-4 / rms) < 1e-12
+
+
+def test_o_graded_error_with_an_output_scale():
+    # s = 10 (dropout p = 0.9): the grade is that of O / s, with the output's own half ulp
+    ref = np.array([0.5, 2.5, 30.0])
+    assert o_graded_error(ref + 0.05, ref, torch.bfloat16, 10.0) == 0.005 or \
+        abs(o_graded_error(ref + 0.05, ref, torch.bfloat16, 10.0) - 0.005) < 1e-12
+    assert o_graded_error(ref + 0.11, ref, torch.bfloat16, 10.0) > O_ATOL
+    # at |O| = 30 (bf16 spacing 0.125) exact rounding passes
+    out = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+    assert o_graded_error(out, ref, torch.bfloat16, 10.0) <= O_ATOL

@@ -4,8 +4,11 @@ Some hosts of this library (plugins inside an engine that owns all device memory
 loops that forbid cudaMalloc after start-up) can pass inputs and outputs but cannot
 provide the backward pass's scratch workspace.  fa_bwd_noalloc takes that scratch from a
 static array inside the library instead.  This test calls it through the C ABI and checks
-that two calls in a row give the results of fa_bwd with a caller-allocated workspace, and
-that a problem too large for the static array is refused without doing any work.
+that two calls in a row give the results of fa_bwd with a caller-allocated workspace
+(dK and dV bit for bit, dQ up to the order of its fp32 reductions) and match the fp64
+oracle within the parity tolerances; that a call allocates no device memory; that the
+largest problem the array accepts runs correctly; and that a problem too large for the
+array is refused without doing any work.
 
 The file is named so that pytest collects it last: if it fails, a run that stops at the
 first failure has already run every other test.  It passes on its own in a fresh process
@@ -18,7 +21,13 @@ import torch
 
 from exact_io_aware_60_b200 import fa
 from exact_io_aware_60_b200 import workloads as W
-from parity import GRAD_REL_L2, rel_l2
+from parity import GRAD_REL_L2, compare_backward, oracle_full, rel_l2
+
+# dQ is summed into fp32 by reductions whose order varies between runs (up to hundreds of
+# key tiles per query tile here); a last-bit difference of the fp32 sum flips the 16-bit
+# output by one ulp (2^-8 relative in bf16) when it lies near a rounding boundary, so two
+# runs differ by about 1e-5 in relative L2.  dK and dV are accumulated in a fixed order.
+DQ_REPEAT_REL_L2 = 1e-4
 
 pytestmark = pytest.mark.gpu
 
@@ -43,11 +52,9 @@ def call_noalloc(L, t, w, out):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
-def test_noalloc_matches_workspace_entry_point_on_two_calls(w):
-    L = fa.lib()
+def device_tensors(w, seed):
     dev = torch.device("cuda", 0)
-    inp = W.make_inputs(w, seed=77)
+    inp = W.make_inputs(w, seed=seed)
     t = {n: inp[n].to(dev) for n in ("q", "k", "v", "do")}
     t["kv_len"] = None if inp["kv_len"] is None else inp["kv_len"].to(dev)
     t["o"], t["lse"] = fa.forward(t["q"], t["k"], t["v"], scale=w.scale, causal=w.causal,
@@ -56,15 +63,60 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(w):
                    fa.backward(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], scale=w.scale,
                                causal=w.causal, kv_len=t["kv_len"])))
     torch.cuda.synchronize()
+    return inp, t, ref
+
+
+def check_against_workspace_call(out, ref, call):
+    assert torch.equal(out["dk"], ref["dk"]) and torch.equal(out["dv"], ref["dv"]), call
+    err = rel_l2(out["dq"].double().cpu().numpy(), ref["dq"].double().cpu().numpy())
+    assert err <= DQ_REPEAT_REL_L2, (call, err)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_noalloc_matches_workspace_entry_point_on_two_calls(w):
+    L = fa.lib()
+    inp, t, ref = device_tensors(w, seed=77)
+    oracle_ref = oracle_full(inp, w.scale, w.causal)
     for call in range(2):
         # start from garbage so that stale outputs cannot pass
         out = {n: torch.full_like(t["q"], float("nan")) for n in ("dq", "dk", "dv")}
         assert call_noalloc(L, t, w, out) == fa.FA_OK
         torch.cuda.synchronize()
         assert fa.fa_get_device_status() == fa.FA_OK
-        for n in ("dq", "dk", "dv"):
-            err = rel_l2(out[n].double().cpu().numpy(), ref[n].double().cpu().numpy())
-            assert err <= GRAD_REL_L2, (call, n, err)
+        check_against_workspace_call(out, ref, call)
+        g = compare_backward({n: out[n].cpu() for n in out}, oracle_ref)
+        assert max(g.values()) <= GRAD_REL_L2, (call, g)
+
+
+def test_noalloc_call_allocates_no_device_memory():
+    L = fa.lib()
+    w = CASES[0]
+    _, t, _ = device_tensors(w, seed=5)
+    out = {n: torch.empty_like(t["q"]) for n in ("dq", "dk", "dv")}
+    assert call_noalloc(L, t, w, out) == fa.FA_OK  # first call: module and symbol set-up
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    assert call_noalloc(L, t, w, out) == fa.FA_OK
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before
+    assert fa.fa_get_device_status() == fa.FA_OK
+
+
+def test_noalloc_largest_accepted_problem():
+    """B*H*N = 254080 rows at d = 64 (N a multiple of 128) is the largest problem whose
+    scratch fits the static array; 128 more rows would not."""
+    L = fa.lib()
+    w = W.custom("limit", B=1, H=5, N=50816, d=64, dtype=torch.bfloat16, causal=True)
+    assert L.fa_bwd_workspace_bytes(w.B, w.H, w.N, w.d) <= fa.FA_NOALLOC_SCRATCH_BYTES
+    assert L.fa_bwd_workspace_bytes(w.B, w.H, w.N + 128, w.d) > fa.FA_NOALLOC_SCRATCH_BYTES
+    _, t, ref = device_tensors(w, seed=9)
+    for call in range(2):
+        out = {n: torch.full_like(t["q"], float("nan")) for n in ("dq", "dk", "dv")}
+        assert call_noalloc(L, t, w, out) == fa.FA_OK
+        torch.cuda.synchronize()
+        assert fa.fa_get_device_status() == fa.FA_OK
+        check_against_workspace_call(out, ref, call)
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
