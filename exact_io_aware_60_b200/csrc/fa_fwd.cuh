@@ -10,9 +10,11 @@
 // B200 mapping: persistent CTAs (two per SM at d = 64), each walking a static list of
 // work items = 128-row query tiles of one (batch, head) (and one key range in split-KV
 // mode).  Per CTA:
-//   warp 4      TMA producer: Q of an item once the previous item's last S MMA is done,
-//               then K_j / V_j into an NS-stage shared-memory ring (128-byte swizzle,
-//               mbarrier transaction counts) that runs on across items.
+//   warp 4      TMA producer: Q of an item (two buffers at d = 64, so the next item's Q
+//               is loaded while this one runs; one at d = 128, loaded once the previous
+//               item's last S MMA is done), then K_j / V_j into an NS-stage shared-memory
+//               ring (128-byte swizzle, mbarrier transaction counts) that runs on across
+//               items.
 //   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM, then O += P_j V_j with
 //               P_j read straight from TMEM.
 //   warps 0..3  softmax, one query row per thread (TMEM lane = row): load S_j, mask on
@@ -95,13 +97,15 @@ struct FwdCfg {
     static constexpr bool P_OWN = (D == 64);            // P in its own TMEM columns
     static constexpr int SBUF = (D == 64) ? 1 : 2;      // score buffers in TMEM
     static constexpr int CTAS_PER_SM = (D == 64) ? 2 : 1;
-    static constexpr int NS = (D == 64) ? 4 : 2;        // K/V ring depth
+    // d = 64: two Q buffers and a 3-deep K/V ring fit two CTAs in an SM's shared memory
+    static constexpr int QBUF = (D == 64) ? 2 : 1;      // Q buffers (items in flight)
+    static constexpr int NS = (D == 64) ? 3 : 2;        // K/V ring depth
     // Each V stage is followed by a block of 16-bit ones, one 64-column block past the
     // tile: the PV MMA reads it as B columns D..D+15 and so also produces the row sums
     // of P (one N = D + 16 instruction instead of a second, equally costly N = 16 one).
     static constexpr int VSTAGE = (HALVES + 1) * KHALF;  // V block + its ones block
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + QTILE;
+    static constexpr int OFF_K = OFF_Q + QBUF * QTILE;
     static constexpr int OFF_V = OFF_K + NS * KTILE;
     static constexpr int OFF_BAR = OFF_V + NS * VSTAGE;
     static constexpr int USED = OFF_BAR + 256;
@@ -119,6 +123,8 @@ struct FwdCfg {
     static constexpr int KS_PV = BN / 16;               // MMA K steps of P V
     static constexpr int PV_STEP = 16 * 128;            // bytes of V rows per P V step
     static_assert(COL_SUM + 16 <= TMEM_COLS, "TMEM budget");
+    // (an SM has 228 KB of shared memory and reserves 1 KB per resident CTA)
+    static_assert(CTAS_PER_SM * (SMEM + 1024) <= 233472, "shared memory budget");
 };
 
 // E4M3 inputs, d = 128: a row of Q, K or V is one 128-byte swizzle block, an MMA step
@@ -135,6 +141,7 @@ struct FwdCfgF8 {
     static constexpr bool P_OWN = false;
     static constexpr int SBUF = 2;
     static constexpr int CTAS_PER_SM = 1;
+    static constexpr int QBUF = 1;
     static constexpr int NS = 4;
     static constexpr int VSTAGE = 2 * KHALF;            // V block + its block of E4M3 ones
     static constexpr int OFF_Q = 0;
@@ -159,8 +166,8 @@ struct FwdCfgF8 {
 };
 
 struct FwdBars {
-    uint64_t q_full;
-    uint64_t q_empty;  // every S MMA of the current item is done: Q may be reloaded
+    uint64_t q_full[2];
+    uint64_t q_empty[2];  // every S MMA of the item in this Q buffer is done: it may be reloaded
     uint64_t o_empty;  // the epilogue has read O: the next item's first P V may start
     uint64_t s_full[2];
     uint64_t s_read;
@@ -196,6 +203,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
     FwdBars *bars = reinterpret_cast<FwdBars *>(smem + C::OFF_BAR);
+    static_assert(sizeof(FwdBars) <= 256, "barrier area");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -204,8 +212,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
-        mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->q_full[i], 1);
+            mbar_init(&bars->q_empty[i], 1);
+        }
         mbar_init(&bars->o_empty, 128);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
@@ -291,10 +301,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             Item it;
             for (int r = 0; ok && item_at(r, it); ++r) {
                 if (it.j_first >= it.T) continue;
-                if (t > 0 && !mbar_wait(&bars->q_empty, (t - 1) & 1)) break;
-                mbar_arrive_expect_tx(&bars->q_full, C::QTILE);
+                // Q buffer qb: the item QBUF back has issued its last S MMA
+                const int qb = t % C::QBUF;
+                if (t >= C::QBUF && !mbar_wait(&bars->q_empty[qb], ((t / C::QBUF) - 1) & 1)) break;
+                mbar_arrive_expect_tx(&bars->q_full[qb], C::QTILE);
                 for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_3d(sQ + hf * C::QHALF, &tmQ, &bars->q_full, hf * 64, it.qt * C::BM, it.bh);
+                    tma_load_3d(sQ + qb * C::QTILE + hf * C::QHALF, &tmQ, &bars->q_full[qb], hf * 64,
+                                it.qt * C::BM, it.bh);
                 for (int j = it.j_first; j < it.T; j = next_block(it, j + 1), ++gj) {
                     const int s = gj % C::NS;
                     if (gj >= C::NS && !mbar_wait(&bars->kv_empty[s], ((gj / C::NS) - 1) & 1)) {
@@ -322,7 +335,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                             : idesc_f16(BF16, false, true, 128, C::PV_N);
             // Descriptors are built once; per k-step and per stage only the 16-byte start
             // address field changes, by compile-time offsets.
-            const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t q_desc0 = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            uint64_t q_desc = q_desc0;  // the current item's Q buffer
             const uint64_t k_desc = smem_desc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t v_desc = smem_desc_sw128(smem_u32(sV), C::KHALF, 1024);
             // g: global block index (stages, phases and score buffers follow it)
@@ -347,8 +361,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             Item it;
             for (int r = 0; ok && item_at(r, it); ++r) {
                 if (it.j_first >= it.T) continue;
-                if (!mbar_wait(&bars->q_full, t & 1)) break;
+                const int qb = t % C::QBUF;
+                if (!mbar_wait(&bars->q_full[qb], (t / C::QBUF) & 1)) break;
                 tc_fence_after();
+                q_desc = q_desc0 + (uint64_t)((qb * C::QTILE) >> 4);
                 // The item's first S overwrites the previous block's S once the softmax has
                 // read it (d = 64); at d = 128 its buffer held P_{g-2}, consumed by an
                 // earlier P V.
@@ -366,7 +382,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             if (!issue_s(g + 1)) { ok = false; break; }  // other buffer is free
                         }
                     } else {
-                        mma_commit(&bars->q_empty);  // every S of the item is issued: Q is free
+                        mma_commit(&bars->q_empty[qb]);  // every S of the item is issued: Q is free
                     }
                     const int s = g % C::NS;
                     if (!mbar_wait(&bars->p_full[g % C::SBUF], (g / C::SBUF) & 1) ||
