@@ -214,7 +214,6 @@ struct BwdBars {
     uint64_t do_full[3];
     uint64_t stage_empty[3];
     uint64_t dq_stage_free;  // d = 128: the dQ drain has finished with the dS buffer
-    uint64_t dp_read;  // d = 64: every P/dS warp has read dP^T (its columns may take the next)
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
         dkv_full, dkv_empty;
     uint32_t tmem_base;
@@ -278,7 +277,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bars->p_full, 256);
         mbar_init(&bars->p_free, 1);
         mbar_init(&bars->ds_full, 256);
-        mbar_init(&bars->dp_read, 256);
         mbar_init(&bars->ds_empty, 1);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 128);
@@ -429,30 +427,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if (C::P_OWN && gi > 0 && !mbar_wait(&bars->s_free, (gi - 1) & 1)) break;
                     if (!mbar_wait(&bars->q_full[s0], (gi / C::QS) & 1)) break;
                     tc_fence_after();
-                    if (D == 64) {
-                        // S^T and dP^T as two interleaved chains (MMAs into one accumulator
-                        // run one after the other; independent ones overlap)
-                        if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
-                            mma_ss(tmem + C::COL_S, k_kmaj + off, q_kmaj + stage_off(s0) + off, kIdescSq,
-                                   kk > 0 ? 1u : 0u);
-                            mma_ss(tmem + C::COL_DP, v_kmaj + off, do_kmaj + stage_off(s0) + off, kIdescSq,
-                                   kk > 0 ? 1u : 0u);
-                        }
-                        mma_commit(&bars->s_full);
-                        mma_commit(&bars->dp_full);
-                    } else {
-                        mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s0));
-                        mma_commit(&bars->s_full);
-                        if (gi > 0 && !mbar_wait(&bars->dq_empty, (gi - 1) & 1)) break;
-                        if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
-                        tc_fence_after();
-                        mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s0));
-                        mma_commit(&bars->dp_full);
-                    }
+                    mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s0));
+                    mma_commit(&bars->s_full);
+                    if (D == 128 && gi > 0 && !mbar_wait(&bars->dq_empty, (gi - 1) & 1)) break;
+                    if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
+                    tc_fence_after();
+                    mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s0));
+                    mma_commit(&bars->dp_full);
                 }
                 for (int i = 0; i < n; ++i) {
                     const int g = gi + i;  // global iteration: ring stage and barrier phases
@@ -474,15 +455,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE,
                                do_mn + stage_off(s), i > 0);
                     mma_commit(&bars->p_free);
-                    if (D == 64 && i + 1 < n) {
-                        // dS^T_i goes to the P^T columns, so dP^T_{i+1} may overwrite dP^T_i
-                        // as soon as every P/dS warp has read it, ahead of dK_i and dQ_i.
-                        if (!mbar_wait(&bars->dp_read, g & 1) ||
-                            !mbar_wait(&bars->do_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
-                        tc_fence_after();
-                        mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
-                        mma_commit(&bars->dp_full);
-                    }
                     if (!C::P_OWN && i + 1 < n) {
                         // P^T_i lives in the S^T columns: S_{i+1} follows dV_i.
                         if (!mbar_wait(&bars->q_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
@@ -492,34 +464,24 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                     if (!mbar_wait(&bars->ds_full, g & 1)) { ok = false; break; }
                     tc_fence_after();
-                    if (D == 64) {
-                        // dK_i and dQ_i as two interleaved chains (dQ has columns of its own)
-                        if (g > 0 && !mbar_wait(&bars->dq_empty, (g - 1) & 1)) { ok = false; break; }
+                    mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
+                               q_mn + stage_off(s), i > 0);
+                    if (D == 64 && g > 0) {
+                        if (!mbar_wait(&bars->dq_empty, (g - 1) & 1)) { ok = false; break; }
                         tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            mma_ts(tmem + C::COL_DK,  // dS^T_i from the P^T columns
-                                   tmem + C::COL_P + (kk >> 2) * C::P_HALF_STRIDE + (kk & 3) * 8,
-                                   q_mn + stage_off(s) + (uint64_t)(kk * 2048 >> 4), kIdescTs,
-                                   (i > 0 || kk > 0) ? 1u : 0u);
-                            mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
-                                   k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
-                        }
-                    } else {
-                        // dQ is written over dS^T, which dK reads: dK first
-                        mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
-                                   q_mn + stage_off(s), i > 0);
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
-                                   k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
                     }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
+                               k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
                     mma_commit(&bars->dq_full);
                     mma_commit(&bars->ds_empty);
                     mma_commit(&bars->stage_empty[s]);
-                    if (D == 128 && i + 1 < n) {
-                        // dQ_i lives in the dP^T columns: wait until it has been drained.
-                        if (!mbar_wait(&bars->dq_empty, g & 1)) { ok = false; break; }
+                    if (i + 1 < n) {
+                        if (D == 128) {
+                            // dQ_i lives in the dP^T columns: wait until it has been drained.
+                            if (!mbar_wait(&bars->dq_empty, g & 1)) { ok = false; break; }
+                        }
                         if (!mbar_wait(&bars->do_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
                         tc_fence_after();
                         mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
@@ -640,23 +602,19 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mbar_arrive(&bars->s_free);  // S^T may now be overwritten by S_{i+1}
                 }
                 const float *nl2 = sLSE + s * 128 + h * 64;  // -LSE2 of the 64 queries
-                const float2 sl2x2 = make_float2(sl2, sl2);
                 // Masks only on the causal diagonal tile and the key-padding tail tile.
                 const bool diag = p.causal && (qi == kt);
                 const bool tile_masked = diag || (kt * 128 + 128 > L);
                 if (!tile_masked) {
-                    // the exponent argument as one packed fused multiply-add per pair
 #pragma unroll
                     for (int k = 0; k < 64; k += 4) {
                         const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k);
-                        const float2 x01 = __ffma2_rn(
-                            make_float2(__uint_as_float(w[k]), __uint_as_float(w[k + 1])), sl2x2,
-                            make_float2(l4.x, l4.y));
-                        const float2 x23 = __ffma2_rn(
-                            make_float2(__uint_as_float(w[k + 2]), __uint_as_float(w[k + 3])), sl2x2,
-                            make_float2(l4.z, l4.w));
-                        Pw[k >> 1] = pack2<BF16>(ex2(x01.x), ex2(x01.y));
-                        Pw[(k >> 1) + 1] = pack2<BF16>(ex2(x23.x), ex2(x23.y));
+                        const float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, l4.x));
+                        const float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, l4.y));
+                        const float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, l4.z));
+                        const float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, l4.w));
+                        Pw[k >> 1] = pack2<BF16>(p0, p1);
+                        Pw[(k >> 1) + 1] = pack2<BF16>(p2, p3);
                     }
                 } else {
 #pragma unroll
@@ -677,10 +635,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                 }
             }
-            // d = 64: the P^T columns last held dS^T_{g-1}: dK_{g-1} (issued after dV_{g-1})
-            // must have read it
-            if (C::P_OWN && g > 0 &&
-                !__all_sync(0xffffffffu, mbar_wait(&bars->ds_empty, (g - 1) & 1))) {
+            if (C::P_OWN && g > 0 &&  // dV_{g-1} has read P
+                !__all_sync(0xffffffffu, mbar_wait(&bars->p_free, (g - 1) & 1))) {
                 ok = false;
                 break;
             }
@@ -714,16 +670,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const float *ndv = sDv + s * 128 + h * 64;  // -D of the 64 queries
             uint32_t wdp[64];
             tmem_ld64(tmem + lane_base + C::COL_DP + h * 64, wdp);
-            if (C::P_OWN) {
-                tc_fence_before();
-                mbar_arrive(&bars->dp_read);  // dP^T may now be overwritten by dP^T_{g+1}
-                // dS^T goes over P^T, which dV_g must have read
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars->p_free, g & 1))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-            }
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const uint32_t *w = wdp + cc * 32;
@@ -737,17 +683,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (!((kb[cc] >> (k >> 1)) & 1u)) dp0 = 0.f;
                         if (!((kb[cc] >> ((k >> 1) + 16)) & 1u)) dp1 = 0.f;
                     }
-                    // dS = P o (dP - D): the difference in fp32 (one packed add), rounded to
-                    // 16 bits, times the 16-bit P pair in one packed multiply
-                    const float2 diff = __fadd2_rn(make_float2(dp0, dp1), nd2);
-                    pk[k >> 1] = mul2<BF16>(Pw[cc * 16 + (k >> 1)], pack2<BF16>(diff.x, diff.y));
+                    // dS = P o (dP - D): the difference in fp32, rounded to 16 bits, times
+                    // the 16-bit P pair in one packed multiply
+                    pk[k >> 1] = mul2<BF16>(Pw[cc * 16 + (k >> 1)],
+                                            pack2<BF16>(dp0 + nd2.x, dp1 + nd2.y));
                 }
-                // dS^T pairs -> TMEM, the A operand of dK += dS^T Q: over P^T_g at d = 64,
-                // over the dP^T columns this warp has just read at d = 128.
-                if (C::P_OWN)
-                    tmem_st16(tmem + lane_base + C::COL_P + h * C::P_HALF_STRIDE + cc * 16, pk);
-                else
-                    tmem_st16(tmem + lane_base + C::COL_DP + h * C::DS_HALF_STRIDE + cc * 16, pk);
+                // dS^T pairs -> TMEM, over dP^T columns this warp has just read; A operand
+                // of dK += dS^T Q.
+                tmem_st16(tmem + lane_base + C::COL_DP + h * C::DS_HALF_STRIDE + cc * 16, pk);
                 // dS -> shared memory as the MN-major A operand of dQ = dS K:
                 // [query block h (64 queries)][key row t][128 bytes], 128-byte swizzle.
                 uint8_t *rowp = sdS + h * 16384 + t * 128;
