@@ -138,9 +138,6 @@ KERNEL_SOURCES = {
     "fa_bwd_kernel": (("fa_bwd.cuh", "sm100.cuh", "dropout.cuh"),
                       ("launch_bwd", "bwd_workspace_layout", "make_map", "launch_pdl",
                        "set_smem", "grid_for")),
-    "fa_bwd64_kernel": (("fa_bwd64.cuh", "fa_bwd.cuh", "sm100.cuh", "dropout.cuh"),
-                        ("launch_bwd", "bwd_workspace_layout", "make_map", "launch_pdl",
-                         "set_smem", "grid_for")),
 }
 
 
@@ -211,7 +208,8 @@ def profile_traffic(kernel: str, workload: str):
     if vals.get("source_sha") != kernel_source_sha(kernel):
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        # (a scaled capture states its factor after the number)
+        return float(vals["dram_bytes_per_launch"].split()[0])
     except (KeyError, ValueError):
         return None
 
@@ -415,16 +413,6 @@ def cpu_baseline_sample(w, inp, budget_s: float, dropout_p: float = 0.0, fp8_set
                       + f" in {dt:.1f} s (nominal FLOPs)"}
 
 
-def bwd_kernel_name(w, args) -> str:
-    """The backward main kernel a measured path launches (the library's rule): the
-    four-issuer kernel at d = 64 without dropout when a key tile visits at least 16 query
-    tiles on average (half of them under causal masking), else the general kernel."""
-    tiles = (w.N + 127) // 128
-    mean_q_tiles = (tiles + 1) // 2 if w.causal else tiles
-    use64 = w.d == 64 and args.dropout == 0 and mean_q_tiles >= 16
-    return "fa_bwd64_kernel" if use64 else "fa_bwd_kernel"
-
-
 def config_dict(w, args, world: int) -> dict:
     """The workload description both arms print (identical for the same flags)."""
     mask = local_global_mask((w.N + 127) // 128) if args.block_sparse else None
@@ -514,7 +502,7 @@ def measure_other_workload(name, dev, stream, steps, peak, hbm, args):
     k_f = sum(x.elapsed_time(y) for x, y in evs[0]) / steps
     k_b = sum(x.elapsed_time(y) for x, y in evs[1]) / steps
     tf = lambda f, ms: f / (ms * 1e-3) / 1e12
-    fk, bk = "fa_fwd_kernel", bwd_kernel_name(w, args)
+    fk, bk = "fa_fwd_kernel", "fa_bwd_kernel"
     res = {"workload": w.description, "steps": steps, "inputs_sets": nsets,
            "ms_per_step": step_ms, "tflops_step": tf(f_fwd + f_bwd, step_ms),
            fk: {"ms": k_f, "tflops": tf(f_fwd, k_f), "frac": tf(f_fwd, k_f) / peak},
@@ -618,7 +606,7 @@ def bench_ours(args, rank, world, local_rank):
         ts = sorted(a.elapsed_time(b) for a, b in pairs)
         pick = lambda q: ts[min(len(ts) - 1, int(q * (len(ts) - 1) + 0.5))]
         return {"calls": len(ts), "median_ms": pick(0.5), "p10_ms": pick(0.1), "p90_ms": pick(0.9)}
-    fwd_name, bwd_name = "fa_fwd_kernel", bwd_kernel_name(w, args)
+    fwd_name, bwd_name = "fa_fwd_kernel", "fa_bwd_kernel"
     per_call = {fwd_name: spread(evs[0])}
     if not fwd_only:
         per_call[bwd_name] = spread(evs[1])

@@ -17,7 +17,6 @@
 #include "fa.h"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
-#include "fa_bwd64.cuh"
 
 namespace {
 
@@ -218,13 +217,6 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
 }
 
 
-// The d = 64 backward pass (without dropout) uses fa_bwd64_kernel when a key tile visits at
-// least this many 128-row query tiles on average.  Measured on B200 (general kernel vs
-// fa_bwd64_kernel, whole backward pass): 4 tiles (N 1024 causal) 87.5 vs 95.5 us, 8 (N 2048
-// causal) 129 vs 137 us, 16 (N 2048 dense) 230 vs 209 us, 16 (N 4096 causal) 211 vs 213 us,
-// 32 (N 4096 dense) 422 vs 382 us, 64 (N 8192 dense) 806 vs 727 us.
-constexpr int kBwd64MinQueryTiles = 16;
-
 struct BwdWorkspace {
     float *dq_acc;
     float *nlse2;
@@ -318,19 +310,9 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.drop = drop;
     p.dv_mul = drop.keep_scale;
     p.dk_mul = scale * drop.keep_scale;
-    p.dk = dk;
-    p.dv = dv;
-    // d = 64 without dropout, long sequences: the kernel whose products have four issuing
-    // threads (fa_bwd64.cuh) is faster per (key tile, query tile) step but slower to start
-    // and finish a key tile, so it is used when a key tile visits at least
-    // kBwd64MinQueryTiles query tiles on average (half the tiles under causal masking).
-    const int mean_q_tiles = causal ? (num_tiles + 1) / 2 : num_tiles;
-    const bool use64 = (D == 64 && !DROP) && mean_q_tiles >= kBwd64MinQueryTiles;
-    auto kern = use64 ? fa::fa_bwd64_kernel<BF16> : fa::fa_bwd_kernel<D, BF16, DROP>;
-    const int threads = use64 ? fa::Bwd64Cfg::THREADS : C::THREADS;
-    const int smem = use64 ? fa::Bwd64Cfg::SMEM : C::SMEM;
-    static std::atomic<int> smem_done[2][kMaxDevices];
-    e = set_smem(kern, smem, smem_done[use64 ? 1 : 0], dev);
+    auto kern = fa::fa_bwd_kernel<D, BF16, DROP>;
+    static std::atomic<int> smem_done[kMaxDevices];
+    e = set_smem(kern, C::SMEM, smem_done, dev);
     if (e != cudaSuccess) {
         record_cuda_error(e, "cudaFuncSetAttribute(bwd)");
         return FA_ERR_CUDA;
@@ -344,7 +326,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         sms = 148;
     const long long grid = std::min<long long>(items, sms);
     timing_mark(1, 0, st);
-    e = launch_pdl(kern, dim3((unsigned)grid), dim3(threads), smem, st, mq, mk, mv, mdo,
+    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mdo,
                    mdk, mdv, mdq, p);
     if (e == cudaSuccess) e = cudaGetLastError();
     timing_mark(1, 1, st);

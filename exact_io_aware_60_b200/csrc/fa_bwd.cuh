@@ -143,8 +143,6 @@ struct BwdParams {
     long long bmask_bh_stride;  // 0: one mask for every (batch, head)
     const float *ndvec;  // [BH][Npad], -D
     float *dq_acc;      // [BH][N][D] fp32
-    void *dk;           // [BH][N][D] 16-bit outputs (written from registers by the d = 64
-    void *dv;           // kernel; the general kernel stores them through TMA maps)
     const int *kv_len;
     int N;
     int Npad;

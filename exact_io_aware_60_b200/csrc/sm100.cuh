@@ -490,35 +490,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x of two values on the FMA pipe instead of the MUFU (which computes one exponential
-// per lane every four cycles per SM sub-partition and is the scarcest unit of a d = 64
-// softmax).  Range reduction in the manner of Cody and Waite: x = n + f with n = round(x),
-// found by adding 1.5 * 2^23 so that n lands in the low mantissa bits, and f in [-1/2, 1/2];
-// 2^f from a degree-3 polynomial whose coefficients minimise the largest relative error on
-// [-1/2, 1/2] (Remez exchange: 7.5e-5, i.e. 13.7 bits, well inside the 8 bits a 16-bit P
-// keeps); 2^n is then added to the exponent field.  x is clamped to >= -125 so that the
-// result stays a normal number (it is then about 2^-125, i.e. zero for every use here).
-constexpr float kExp2C0 = 0.99992807354f;
-constexpr float kExp2C1 = 0.69326098546f;
-constexpr float kExp2C2 = 0.24261112219f;
-constexpr float kExp2C3 = 0.05517166906f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 t = __fadd2_rn(x, make_float2(kRoundMagic, kRoundMagic));
-    const float2 n = __fadd2_rn(t, make_float2(-kRoundMagic, -kRoundMagic));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);  // exact: x - n
-    float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-    p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
-    p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
-    // the low 9 bits of t's encoding are n (two's complement): shifted into the exponent
-    const uint32_t rx = __float_as_uint(t.x) * 8388608u + __float_as_uint(p.x);
-    const uint32_t ry = __float_as_uint(t.y) * 8388608u + __float_as_uint(p.y);
-    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
-}
-
 // max of three floats in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;

@@ -35,7 +35,7 @@ CASES = [
     (1, 2, 1024, 64, torch.bfloat16, False, None, True, 0.3, 3),
     (1, 2, 640, 128, torch.bfloat16, True, None, False, 0.7, 4),
     (3, 1, 256, 64, torch.float16, False, (30, 256), False, 0.6, 5),
-    # d = 64 from 4096 rows: the four-issuer backward kernel
+    # d = 64 with 33 tiles per side, causal and key-padded
     (1, 1, 4173, 64, torch.bfloat16, True, None, False, 0.4, 6),
     (2, 1, 4224, 64, torch.float16, False, (1000, 4224), True, 0.3, 7),
 ]

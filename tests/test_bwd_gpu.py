@@ -47,8 +47,8 @@ def test_backward_edge_shapes(N, d, dtype, causal, kvr):
             assert torch.all(gpu["dk"][b, :, L:] == 0) and torch.all(gpu["dv"][b, :, L:] == 0)
 
 
-# d = 64 from 4096 rows up runs the four-issuer backward kernel: ragged tails, causal
-# masking, key padding (including an empty sequence) at that size.
+# d = 64 at 4096 rows and more (32+ query tiles per head): ragged tails, causal masking,
+# key padding (including an empty sequence).
 LONG_EDGE = [
     # (N, dtype, causal, kv_len_range)
     (4096, torch.bfloat16, True, None),
