@@ -593,45 +593,53 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             // (exactly what the dV MMA consumes; dS below uses the same rounded values).
             uint32_t Pw[32];
             {
-                uint32_t w[64];
-                tmem_ld64(tmem + lane_base + C::COL_S + h * 64, w);
-                if (C::P_OWN) {
-                    tc_fence_before();
-                    mbar_arrive(&bars->s_free);  // S^T may now be overwritten by S_{i+1}
-                }
                 const float *nl2 = sLSE + s * 128 + h * 64;  // -LSE2 of the 64 queries
                 // Masks only on the causal diagonal tile and the key-padding tail tile.
                 const bool diag = p.causal && (qi == kt);
                 const bool tile_masked = diag || (kt * 128 + 128 > L);
-                if (!tile_masked) {
+                // P^T for queries 64h + k0 .. + 31 from the S^T values w
+                auto p_half = [&](const uint32_t (&w)[32], int k0) {
+                    if (!tile_masked) {
 #pragma unroll
-                    for (int k = 0; k < 64; k += 4) {
-                        const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k);
-                        const float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, l4.x));
-                        const float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, l4.y));
-                        const float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, l4.z));
-                        const float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, l4.w));
-                        Pw[k >> 1] = pack2<BF16>(p0, p1);
-                        Pw[(k >> 1) + 1] = pack2<BF16>(p2, p3);
-                    }
-                } else {
+                        for (int k = 0; k < 32; k += 4) {
+                            const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k0 + k);
+                            const float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, l4.x));
+                            const float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, l4.y));
+                            const float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, l4.z));
+                            const float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, l4.w));
+                            Pw[(k0 + k) >> 1] = pack2<BF16>(p0, p1);
+                            Pw[((k0 + k) >> 1) + 1] = pack2<BF16>(p2, p3);
+                        }
+                    } else {
 #pragma unroll
-                    for (int k = 0; k < 64; k += 4) {
-                        const int c = h * 64 + k;  // query column in the tile
-                        const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k);
-                        float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, l4.x));
-                        float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, l4.y));
-                        float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, l4.z));
-                        float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, l4.w));
-                        // keys past the valid length, and queries before the key (causal)
-                        if (!key_ok || (diag && c < t)) p0 = 0.f;
-                        if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
-                        if (!key_ok || (diag && c + 2 < t)) p2 = 0.f;
-                        if (!key_ok || (diag && c + 3 < t)) p3 = 0.f;
-                        Pw[k >> 1] = pack2<BF16>(p0, p1);
-                        Pw[(k >> 1) + 1] = pack2<BF16>(p2, p3);
+                        for (int k = 0; k < 32; k += 4) {
+                            const int c = h * 64 + k0 + k;  // query column in the tile
+                            const float4 l4 = *reinterpret_cast<const float4 *>(nl2 + k0 + k);
+                            float p0 = ex2(fmaf(__uint_as_float(w[k]), sl2, l4.x));
+                            float p1 = ex2(fmaf(__uint_as_float(w[k + 1]), sl2, l4.y));
+                            float p2 = ex2(fmaf(__uint_as_float(w[k + 2]), sl2, l4.z));
+                            float p3 = ex2(fmaf(__uint_as_float(w[k + 3]), sl2, l4.w));
+                            // keys past the valid length, and queries before the key (causal)
+                            if (!key_ok || (diag && c < t)) p0 = 0.f;
+                            if (!key_ok || (diag && c + 1 < t)) p1 = 0.f;
+                            if (!key_ok || (diag && c + 2 < t)) p2 = 0.f;
+                            if (!key_ok || (diag && c + 3 < t)) p3 = 0.f;
+                            Pw[(k0 + k) >> 1] = pack2<BF16>(p0, p1);
+                            Pw[((k0 + k) >> 1) + 1] = pack2<BF16>(p2, p3);
+                        }
                     }
+                };
+                // The second half of the S^T row loads while the first is exponentiated.
+                uint32_t wa[32], wb[32];
+                tmem_ld32(tmem + lane_base + C::COL_S + h * 64, wa);
+                tmem_ld32_async(tmem + lane_base + C::COL_S + h * 64 + 32, wb);
+                p_half(wa, 0);
+                tmem_wait_ld(wb);
+                if (C::P_OWN) {
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free);  // S^T may now be overwritten by S_{i+1}
                 }
+                p_half(wb, 32);
             }
             if (C::P_OWN && g > 0 &&  // dV_{g-1} has read P
                 !__all_sync(0xffffffffu, mbar_wait(&bars->p_free, (g - 1) & 1))) {
@@ -666,11 +674,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             tc_fence_after();
             const float *ndv = sDv + s * 128 + h * 64;  // -D of the 64 queries
-            uint32_t wdp[64];
-            tmem_ld64(tmem + lane_base + C::COL_DP + h * 64, wdp);
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const uint32_t *w = wdp + cc * 32;
+            // dS for queries 64h + 32cc .. + 31 from the dP^T values w
+            auto ds_half = [&](const uint32_t (&w)[32], int cc) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
@@ -698,7 +703,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     *reinterpret_cast<uint4 *>(rowp + ((chunk ^ (t & 7)) << 4)) =
                         make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
                 }
-            }
+            };
+            // the second half of the dP^T row loads while the first is turned into dS
+            uint32_t da[32], db[32];
+            tmem_ld32(tmem + lane_base + C::COL_DP + h * 64, da);
+            tmem_ld32_async(tmem + lane_base + C::COL_DP + h * 64 + 32, db);
+            ds_half(da, 0);
+            tmem_wait_ld(db);
+            ds_half(db, 1);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars->ds_full);
