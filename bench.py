@@ -134,10 +134,11 @@ def load_peaks():
 # host function in fa_api.cu that configures and launches it.
 KERNEL_SOURCES = {
     "fa_fwd_kernel": (("fa_fwd.cuh", "sm100.cuh", "dropout.cuh"),
-                      ("launch_fwd", "make_map", "launch_pdl", "set_smem")),
+                      ("launch_fwd", "make_map", "launch_pdl", "set_smem", "balance_items",
+                       "schedule_for", "no_schedule")),
     "fa_bwd_kernel": (("fa_bwd.cuh", "sm100.cuh", "dropout.cuh"),
                       ("launch_bwd", "bwd_workspace_layout", "make_map", "launch_pdl",
-                       "set_smem", "grid_for")),
+                       "set_smem", "grid_for", "balance_items", "schedule_for", "no_schedule")),
 }
 
 

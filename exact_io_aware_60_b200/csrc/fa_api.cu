@@ -11,8 +11,11 @@
 #include <cstdio>
 #include <algorithm>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
+#include <vector>
 
 #include "fa.h"
 #include "fa_fwd.cuh"
@@ -145,6 +148,102 @@ cudaError_t set_smem(K kern, int bytes, std::atomic<int> *done, int dev) {
     return e;
 }
 
+// ---------------------------------------------------------------- static schedules
+
+// Assigns work items 0 .. n-1 with estimated costs `cost` to `lists` persistent CTAs so
+// that the largest list total is small: longest first onto the least loaded list (LPT),
+// then, while it lowers the largest total, moves of an item out of the fullest list and
+// swaps of an item of the fullest list with a smaller one of another list.  Each list is
+// then walked heaviest item first.  Deterministic for given inputs.
+bool balance_items(const std::vector<float> &cost, int lists, fa::ItemSchedule &s) {
+    const int n = (int)cost.size();
+    if (lists < 1 || lists > fa::kSchedMaxLists || n < 1 || n > fa::kSchedMaxItems) return false;
+    std::vector<int> order(n);
+    for (int i = 0; i < n; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+    std::vector<std::vector<int>> bins(lists);
+    std::vector<double> load(lists, 0.0);
+    for (int i : order) {
+        int best = 0;
+        for (int c = 1; c < lists; ++c)
+            if (load[c] < load[best]) best = c;
+        bins[best].push_back(i);
+        load[best] += cost[i];
+    }
+    // (few items per list: there LPT can leave the largest total well above the mean)
+    const int max_iter = (n <= 8 * lists) ? 4 * n : 0;
+    for (int iter = 0; iter < max_iter; ++iter) {
+        int hi = 0;
+        for (int c = 1; c < lists; ++c)
+            if (load[c] > load[hi]) hi = c;
+        bool improved = false;
+        // move: an item of the fullest list to a list that stays below the current maximum
+        for (size_t a = 0; a < bins[hi].size() && !improved; ++a) {
+            const float x = cost[bins[hi][a]];
+            for (int c = 0; c < lists && !improved; ++c)
+                if (c != hi && load[c] + x < load[hi] - 1e-6) {
+                    bins[c].push_back(bins[hi][a]);
+                    bins[hi].erase(bins[hi].begin() + a);
+                    load[c] += x;
+                    load[hi] -= x;
+                    improved = true;
+                }
+        }
+        // swap: an item of the fullest list with a smaller one elsewhere
+        for (size_t a = 0; a < bins[hi].size() && !improved; ++a) {
+            const float x = cost[bins[hi][a]];
+            for (int c = 0; c < lists && !improved; ++c) {
+                if (c == hi) continue;
+                for (size_t b = 0; b < bins[c].size(); ++b) {
+                    const float y = cost[bins[c][b]];
+                    if (y < x && load[c] - y + x < load[hi] - 1e-6) {
+                        std::swap(bins[hi][a], bins[c][b]);
+                        load[hi] += y - x;
+                        load[c] += x - y;
+                        improved = true;
+                        break;
+                    }
+                }
+            }
+        }
+        if (!improved) break;
+    }
+    s.lists = lists;
+    int k = 0;
+    for (int c = 0; c < lists; ++c) {
+        std::stable_sort(bins[c].begin(), bins[c].end(), [&](int a, int b) { return cost[a] > cost[b]; });
+        s.off[c] = (uint16_t)k;
+        for (int i : bins[c]) s.ids[k++] = (uint16_t)i;
+    }
+    s.off[lists] = (uint16_t)k;
+    return true;
+}
+
+// Schedules by problem shape, computed once per shape and kept for the process.
+std::mutex g_sched_mu;
+std::map<std::vector<long long>, fa::ItemSchedule> g_sched;
+
+// The schedule of a shape (lists = 0 when none applies), computed on first use from the
+// items' estimated costs.
+fa::ItemSchedule schedule_for(const std::vector<long long> &key, const std::vector<float> &cost,
+                              int lists) {
+    std::lock_guard<std::mutex> lock(g_sched_mu);
+    auto f = g_sched.find(key);
+    if (f != g_sched.end()) return f->second;
+    fa::ItemSchedule s;
+    std::memset(&s, 0, sizeof(s));
+    if (!balance_items(cost, lists, s)) s.lists = 0;
+    if (g_sched.size() > 256) g_sched.clear();  // bounded cache
+    g_sched.emplace(key, s);
+    return s;
+}
+
+fa::ItemSchedule no_schedule() {
+    fa::ItemSchedule s;
+    std::memset(&s, 0, sizeof(s));
+    return s;
+}
+
 // Split-KV output of one launch: fp32 partial outputs and LSEs (see FwdParams).
 struct SplitOut {
     float *part_o = nullptr;
@@ -191,9 +290,14 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.causal = causal ? 1 : 0;
     p.drop = drop;
     p.out_scale = out_scale;
-    auto kern = fa::fa_fwd_kernel<D, BF16, DROP, SPLIT, F8>;
-    static std::atomic<int> smem_done[kMaxDevices];
-    cudaError_t e = set_smem(kern, C::SMEM, smem_done, dev);
+    // (a scheduled instance exists for the d = 64 forward without key splits only)
+    constexpr bool kCanSched = (D == 64 && !SPLIT && !F8);
+    auto kern = fa::fa_fwd_kernel<D, BF16, DROP, SPLIT, F8, false>;
+    static std::atomic<int> smem_done[2][kMaxDevices];
+    cudaError_t e = set_smem(kern, C::SMEM, smem_done[0], dev);
+    if constexpr (kCanSched)
+        if (e == cudaSuccess)
+            e = set_smem(fa::fa_fwd_kernel<D, BF16, DROP, SPLIT, F8, true>, C::SMEM, smem_done[1], dev);
     if (e != cudaSuccess) {
         record_cuda_error(e, "cudaFuncSetAttribute(fwd)");
         return FA_ERR_CUDA;
@@ -205,8 +309,38 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         sms = 148;
     const long long grid = std::min<long long>(items, (long long)C::CTAS_PER_SM * sms);
+    // Causal shapes (no key lengths or block mask) with several items per CTA: a balanced
+    // static assignment.  Item u is (query tile, head) as the kernel numbers it; its cost
+    // is its key blocks plus a per-item overhead (the epilogue and the next item's first
+    // scores: about 1.8 blocks of 64 keys at d = 64, measured on B200; half that for
+    // 128-key blocks).  Without the causal mask every item costs the same and the zigzag
+    // is already balanced.
+    fa::ItemSchedule sched = no_schedule();
+    if (kCanSched && causal && kv_len == nullptr && bmask == nullptr && items > grid &&
+        items <= fa::kSchedMaxItems) {
+        std::vector<float> cost((size_t)items);
+        for (long long u = 0; u < items; ++u) {
+            const int rank = (int)(u / bh);
+            const int qt = causal ? p.num_q_tiles - 1 - rank : rank;
+            long long kv_end = Nk;
+            if (causal) kv_end = std::min<long long>(kv_end, (long long)(qt + 1) * C::BM + p.causal_off);
+            const long long T = kv_end > 0 ? (kv_end + C::BN - 1) / C::BN : 0;
+            cost[(size_t)u] = (float)T + (C::BN == 64 ? 1.8f : 0.9f);
+        }
+        sched = schedule_for({0, D, N, Nk, bh, causal ? 1 : 0, grid}, cost, (int)grid);
+    }
     timing_mark(0, 0, st);
-    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, p);
+    if constexpr (kCanSched) {
+        if (sched.lists > 0)
+            e = launch_pdl(fa::fa_fwd_kernel<D, BF16, DROP, SPLIT, F8, true>, dim3((unsigned)grid),
+                           dim3(C::THREADS), C::SMEM, st, mq, mk, mv, p, sched);
+        else
+            e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, p,
+                           fa::NoSchedule{0});
+    } else {
+        e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, p,
+                       fa::NoSchedule{0});
+    }
     if (e == cudaSuccess) e = cudaGetLastError();
     timing_mark(0, 1, st);
     if (e != cudaSuccess) {
@@ -310,9 +444,11 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.drop = drop;
     p.dv_mul = drop.keep_scale;
     p.dk_mul = scale * drop.keep_scale;
-    auto kern = fa::fa_bwd_kernel<D, BF16, DROP>;
-    static std::atomic<int> smem_done[kMaxDevices];
-    e = set_smem(kern, C::SMEM, smem_done, dev);
+    auto kern = fa::fa_bwd_kernel<D, BF16, DROP, false>;
+    auto kern_s = fa::fa_bwd_kernel<D, BF16, DROP, true>;
+    static std::atomic<int> smem_done[2][kMaxDevices];
+    e = set_smem(kern, C::SMEM, smem_done[0], dev);
+    if (e == cudaSuccess) e = set_smem(kern_s, C::SMEM, smem_done[1], dev);
     if (e != cudaSuccess) {
         record_cuda_error(e, "cudaFuncSetAttribute(bwd)");
         return FA_ERR_CUDA;
@@ -325,9 +461,28 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         sms = 148;
     const long long grid = std::min<long long>(items, sms);
+    // Causal shapes (no key lengths or block mask) with several items per CTA: a balanced
+    // static assignment.  Item u is (key tile, head) as the kernel numbers it; its cost is
+    // the query tiles it visits plus about 0.9 of one for its epilogue and the next item's
+    // start (measured on B200).  Without the causal mask every item costs the same.
+    fa::ItemSchedule sched = no_schedule();
+    if (causal && kv_len == nullptr && bmask == nullptr && items > grid &&
+        items <= fa::kSchedMaxItems) {
+        std::vector<float> cost((size_t)items);
+        for (long long u = 0; u < items; ++u) {
+            const int kt = (D == 128) ? (int)(u % num_tiles) : (int)(u / bh);
+            const int n = causal ? num_tiles - kt : num_tiles;
+            cost[(size_t)u] = (float)n + 0.9f;
+        }
+        sched = schedule_for({1, D, N, bh, causal ? 1 : 0, grid}, cost, (int)grid);
+    }
     timing_mark(1, 0, st);
-    e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mdo,
-                   mdk, mdv, mdq, p);
+    if (sched.lists > 0)
+        e = launch_pdl(kern_s, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv,
+                       mdo, mdk, mdv, mdq, p, sched);
+    else
+        e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv,
+                       mdo, mdk, mdv, mdq, p, fa::NoSchedule{0});
     if (e == cudaSuccess) e = cudaGetLastError();
     timing_mark(1, 1, st);
     if (e != cudaSuccess) {
@@ -473,6 +628,22 @@ int launch_splitkv(const void *q, const void *k, const void *v, void *o, float *
 extern "C" {
 
 int fa_version(void) { return kVersion; }
+
+int fa_schedule_items(const float *cost, int n, int lists, unsigned short *off,
+                      unsigned short *ids) {
+    if (cost == nullptr || off == nullptr || ids == nullptr) return FA_ERR_INVALID_ARG;
+    if (n < 1 || n > fa::kSchedMaxItems || lists < 1 || lists > fa::kSchedMaxLists)
+        return FA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!(cost[i] > 0.f) || !std::isfinite(cost[i])) return FA_ERR_INVALID_ARG;
+    std::vector<float> c(cost, cost + n);
+    fa::ItemSchedule s;
+    std::memset(&s, 0, sizeof(s));
+    if (!balance_items(c, lists, s)) return FA_ERR_INVALID_ARG;
+    for (int i = 0; i <= lists; ++i) off[i] = s.off[i];
+    for (int i = 0; i < n; ++i) ids[i] = s.ids[i];
+    return FA_OK;
+}
 
 int fa_set_timing_events(int which, void *start, void *stop) {
     if (which < 0 || which > 1) return FA_ERR_INVALID_ARG;

@@ -221,12 +221,14 @@ struct BwdBars {
 //   dV = r (P o K)^T dO,  dP = r K o (dO V^T),  D = rowsum(dO o O),  dS = P o (dP - D);
 // the kernel computes dS' = P o (K o (dO V^T) - D / r) (D / r comes from the preprocess)
 // and folds r into the dV, dK and dQ output multipliers.
-template <int D, bool BF16, bool DROP>
+// SCHED: the launcher passes a static schedule of the items (ItemSchedule).
+template <int D, bool BF16, bool DROP, bool SCHED = false>
 __global__ void __launch_bounds__(448, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
               const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-              const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
+              const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p,
+              const __grid_constant__ std::conditional_t<SCHED, ItemSchedule, NoSchedule> sched) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -253,7 +255,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // d = 128 (head-major: the long-sequence case, where one head's fp32 dQ accumulator
     // should stay in L2).  Round r of CTA c takes item r * G + c on even rounds and
     // r * G + (G - 1 - c) on odd ones (G = grid size); the zigzag evens out the causal
-    // work.  Every role walks the same list on its own.
+    // work.  With a schedule from the launcher (dense and causal shapes of up to
+    // kSchedMaxItems items), CTA c walks its list of items instead.  Every role walks the
+    // same list on its own.
 
     if (warp == C::W_TMA && lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -303,8 +307,15 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         return qi;
     };
     auto item_at = [&](int r, Item &it) -> bool {
-        const int G = (int)gridDim.x;
-        const int u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        int u;
+        if constexpr (SCHED) {  // the launcher's balanced assignment
+            const int b0 = sched.off[blockIdx.x], b1 = sched.off[blockIdx.x + 1];
+            if (r >= b1 - b0) return false;
+            u = sched.ids[b0 + r];
+        } else {
+            const int G = (int)gridDim.x;
+            u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        }
         if (u >= p.num_tiles * p.BH) return false;
         if (D == 128) {
             // head-major: the CTAs of a round share one or two heads, whose fp32 dQ

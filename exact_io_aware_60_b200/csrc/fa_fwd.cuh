@@ -185,10 +185,12 @@ struct FwdBars {
 // normalised by that range's own l) and the range's LSE; a combine kernel merges them.
 // F8: E4M3 Q, K, V (d = 128), kind::f8f6f4 MMAs, P rounded to E4M3 for the P V product,
 // bf16 output (BF16 = true).
-template <int D, bool BF16, bool DROP, bool SPLIT, bool F8 = false>
+// SCHED: the launcher passes a static schedule of the items (ItemSchedule).
+template <int D, bool BF16, bool DROP, bool SPLIT, bool F8 = false, bool SCHED = false>
 __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+              const __grid_constant__ CUtensorMap tmV, const FwdParams p,
+              const __grid_constant__ std::conditional_t<SCHED, ItemSchedule, NoSchedule> sched) {
     static_assert(!F8 || (D == 128 && BF16 && !DROP && !SPLIT), "E4M3 variant: d = 128 only");
     using C = std::conditional_t<F8, FwdCfgF8, FwdCfg<D>>;
     constexpr int BN = C::BN;
@@ -247,9 +249,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     pdl_wait();  // inputs written by the previous kernel are visible from here on
 
     // Persistent CTA: work items are (query tile, key split, head), numbered so that the
-    // heaviest causal tiles come first.  Round r of CTA c takes item r * G + c on even
-    // rounds and r * G + (G - 1 - c) on odd ones (G = grid size).  Every role walks the
-    // same list; key lengths and block masks are read only after the wait above.
+    // heaviest causal tiles come first.  With a schedule from the launcher (dense and
+    // causal shapes of up to kSchedMaxItems items), CTA c walks its list of items;
+    // otherwise round r of CTA c takes item r * G + c on even rounds and r * G + (G - 1 - c)
+    // on odd ones (G = grid size).  Every role walks the same list; key lengths and block
+    // masks are read only after the wait above.
     struct Item {
         int qt, split, bh, L;
         int T;            // end of this item's key-block range
@@ -263,8 +267,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         return j;
     };
     auto item_at = [&](int r, Item &it) -> bool {
-        const int G = (int)gridDim.x;
-        const int u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        int u;
+        if constexpr (SCHED) {  // the launcher's balanced assignment
+            const int b0 = sched.off[blockIdx.x], b1 = sched.off[blockIdx.x + 1];
+            if (r >= b1 - b0) return false;
+            u = sched.ids[b0 + r];
+        } else {
+            const int G = (int)gridDim.x;
+            u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        }
         if (u >= p.num_q_tiles * p.num_splits * p.BH) return false;
         it.bh = u % p.BH;
         const int rest = u / p.BH;

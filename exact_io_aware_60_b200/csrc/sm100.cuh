@@ -100,6 +100,22 @@ __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
     }
 }
 
+// A static assignment of work items to the CTAs of a persistent launch, passed by value
+// as a kernel parameter: CTA c walks items ids[off[c]] .. ids[off[c + 1] - 1] in that
+// order.  lists == 0: no assignment (the kernels walk their zigzag order instead).
+constexpr int kSchedMaxLists = 512;
+constexpr int kSchedMaxItems = 2048;
+struct ItemSchedule {
+    int lists;
+    uint16_t off[kSchedMaxLists + 1];
+    uint16_t ids[kSchedMaxItems];
+};
+// The parameter of a kernel instance that walks its zigzag order (a schedule of 5 KB
+// costs every launch a little even when unused, so such launches use this instead).
+struct NoSchedule {
+    int lists;
+};
+
 // Programmatic dependent launch: kernels of one step are launched so that the next one
 // may start early.  pdl_wait() blocks until the previous kernel in the stream has
 // completed and its memory is visible (it returns at once if there is no such

@@ -96,6 +96,8 @@ def lib():
             L.fa_bwd_noalloc.restype = i
             L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i,
                                          vp, i, vp]
+            L.fa_schedule_items.restype = i
+            L.fa_schedule_items.argtypes = [vp, i, i, vp, vp]
             _lib = L
     return _lib
 
@@ -111,6 +113,20 @@ def fa_strerror(status: int) -> str:
 
 def fa_version() -> int:
     return int(lib().fa_version())
+
+
+def fa_schedule_items(cost, lists: int):
+    """The launchers' static schedule of items with host costs ``cost`` over ``lists``
+    lists: (off, ids) as numpy arrays, list c = ids[off[c]:off[c + 1]] (host only)."""
+    import numpy as np
+    c = np.ascontiguousarray(np.asarray(cost, dtype=np.float32))
+    off = np.zeros(int(lists) + 1, dtype=np.uint16)
+    ids = np.zeros(max(len(c), 1), dtype=np.uint16)
+    rc = lib().fa_schedule_items(c.ctypes.data, len(c), int(lists), off.ctypes.data,
+                                 ids.ctypes.data)
+    if rc != FA_OK:
+        raise FAError(rc, "fa_schedule_items")
+    return off, ids[:len(c)]
 
 
 def _dtype_code(t: torch.Tensor) -> int:

@@ -322,6 +322,17 @@ FA_API int fa_set_timing_events(int which, void *start, void *stop);
  */
 FA_API int fa_selftest_wait_timeout(int limit_us, void *stream);
 
+/* The static schedule the launchers give the persistent kernels for causal shapes with
+ * several work items per CTA (no key lengths, no block mask): items 0 .. n-1 with host
+ * costs cost[i] (> 0) are split over `lists` lists so that the largest list total is small
+ * (longest first onto the least loaded list, then moves and swaps out of the fullest
+ * list); list c is ids[off[c]] .. ids[off[c + 1] - 1], heaviest item first.  Host memory:
+ * cost[n], off[lists + 1], ids[n], all owned by the caller.  Pure host computation (no
+ * GPU, no CUDA call).  FA_ERR_INVALID_ARG for a null pointer, n < 1 or n > 2048, lists < 1
+ * or lists > 512, or a cost that is not a positive finite number. */
+FA_API int fa_schedule_items(const float *cost, int n, int lists, unsigned short *off,
+                             unsigned short *ids);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 FA_API int fa_version(void);
 
