@@ -444,11 +444,16 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.drop = drop;
     p.dv_mul = drop.keep_scale;
     p.dk_mul = scale * drop.keep_scale;
+    // d = 64 without the causal mask: the two-issuer variant (BwdCfg::TWO_ISS).
+    using C2 = fa::BwdCfg<D, true>;
+    const bool two = (D == 64) && !causal;
     auto kern = fa::fa_bwd_kernel<D, BF16, DROP, false>;
     auto kern_s = fa::fa_bwd_kernel<D, BF16, DROP, true>;
-    static std::atomic<int> smem_done[2][kMaxDevices];
+    auto kern_2 = fa::fa_bwd_kernel<D, BF16, DROP, false, D == 64>;
+    static std::atomic<int> smem_done[3][kMaxDevices];
     e = set_smem(kern, C::SMEM, smem_done[0], dev);
     if (e == cudaSuccess) e = set_smem(kern_s, C::SMEM, smem_done[1], dev);
+    if (e == cudaSuccess && two) e = set_smem(kern_2, C2::SMEM, smem_done[2], dev);
     if (e != cudaSuccess) {
         record_cuda_error(e, "cudaFuncSetAttribute(bwd)");
         return FA_ERR_CUDA;
@@ -480,6 +485,9 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     if (sched.lists > 0)
         e = launch_pdl(kern_s, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv,
                        mdo, mdk, mdv, mdq, p, sched);
+    else if (two)
+        e = launch_pdl(kern_2, dim3((unsigned)grid), dim3(C2::THREADS), C2::SMEM, st, mq, mk, mv,
+                       mdo, mdk, mdv, mdq, p, fa::NoSchedule{0});
     else
         e = launch_pdl(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv,
                        mdo, mdk, mdv, mdq, p, fa::NoSchedule{0});

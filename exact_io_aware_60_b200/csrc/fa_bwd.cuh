@@ -23,6 +23,8 @@
 //        warp 9      MMA issuer (one thread), all on tcgen05 with fp32 TMEM accumulators:
 //                    S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i, dK += dS^T Q_i
 //                    (P^T, dS^T read from TMEM), dQ_i = dS K (dS from shared memory).
+//        warp 14     (d = 64 without the causal mask) a second MMA issuer, which takes dK_i
+//                    and dP^T_{i+1} from warp 9 (see BwdCfg::TWO_ISS).
 //        warps 0..7  one key row per thread and half of the query columns per warp
 //                    (lane quarter w % 4, query half w / 4): P^T = 2^(S^T scale log2e -
 //                    LSE2), written back to TMEM as 16-bit pairs; dS^T = P^T o (dP^T - D)
@@ -159,7 +161,8 @@ struct BwdParams {
     float dk_mul;
 };
 
-template <int D>
+// TWO: (d = 64) two MMA-issuing threads instead of one (see TWO_ISS).
+template <int D, bool TWO = false>
 struct BwdCfg {
     static constexpr int TILE = 128 * D * 2;  // one 128-row tile of Q / K / V / dO
     static constexpr int HALF = 128 * 128;    // one 128-byte column block of a tile
@@ -191,8 +194,14 @@ struct BwdCfg {
     static constexpr int SMEM = USED + SLACK;
     // warps 0..7: P / dS (lane quarter w % 4, query half w / 4); 8: TMA; 9: MMA;
     // 10..13: dQ drain (lane quarters 2, 3, 0, 1).
-    static constexpr int THREADS = 448;
-    static constexpr int W_TMA = 8, W_MMA = 9, W_DQ0 = 10;
+    // Two MMA-issuing threads (d = 64, used without the causal mask): A (warp 9) issues S^T,
+    // dV and dQ; B (warp 14) issues dK_i and then dP^T_{i+1}, which overwrites the dS^T_i
+    // that dK_i reads: in one thread's order no completion wait is needed between them.
+    // Measured on B200, this shortens the long items of non-causal shapes by 2-3%, while the
+    // short, uneven items of causal shapes end less evenly across CTAs with it.
+    static constexpr bool TWO_ISS = TWO && (D == 64);
+    static constexpr int THREADS = TWO_ISS ? 480 : 448;
+    static constexpr int W_TMA = 8, W_MMA = 9, W_DQ0 = 10, W_MMA2 = TWO_ISS ? 14 : 9;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0;
     static constexpr uint32_t COL_DP = 128;
@@ -222,14 +231,14 @@ struct BwdBars {
 // the kernel computes dS' = P o (K o (dO V^T) - D / r) (D / r comes from the preprocess)
 // and folds r into the dV, dK and dQ output multipliers.
 // SCHED: the launcher passes a static schedule of the items (ItemSchedule).
-template <int D, bool BF16, bool DROP, bool SCHED = false>
-__global__ void __launch_bounds__(448, 1)
+template <int D, bool BF16, bool DROP, bool SCHED = false, bool TWO = false>
+__global__ void __launch_bounds__(BwdCfg<D, TWO>::THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
               const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
               const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p,
               const __grid_constant__ std::conditional_t<SCHED, ItemSchedule, NoSchedule> sched) {
-    using C = BwdCfg<D>;
+    using C = BwdCfg<D, TWO>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     if (pad > (uint32_t)C::SLACK) {  // cannot happen with a 1024-aligned dynamic base
@@ -271,7 +280,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int i = 0; i < C::QS; ++i) {
             mbar_init(&bars->q_full[i], 1);
             mbar_init(&bars->do_full[i], 1);
-            mbar_init(&bars->stage_empty[i], 1);
+            mbar_init(&bars->stage_empty[i], C::TWO_ISS ? 2 : 1);  // each issuer's last reader
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->s_free, 256);
@@ -283,7 +292,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 128);
         mbar_init(&bars->dq_stage_free, 1);
-        mbar_init(&bars->dkv_full, 1);
+        mbar_init(&bars->dkv_full, C::TWO_ISS ? 2 : 1);  // each issuer's item end
         mbar_init(&bars->dkv_empty, 256);
         fence_mbar_init();
     }
@@ -384,8 +393,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 ++tn;
             }
         }
-    } else if (warp == C::W_MMA) {
-        // ------------------------------ MMA issuer --------------------------------
+    } else if (warp == C::W_MMA || warp == C::W_MMA2) {
+        // ------------------------------ MMA issuers -------------------------------
         if (lane == 0) {
             constexpr uint32_t kIdescSq = idesc_f16(BF16, false, false, 128, 128);  // S^T, dP^T
             constexpr uint32_t kIdescTs = idesc_f16(BF16, false, true, 128, D);     // dV, dK
@@ -422,6 +431,88 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool ok = true;
             int gi = 0, tn = 0;  // global iteration, items with work so far
             Item it;
+            if constexpr (C::TWO_ISS) {
+                const bool is_a = warp == C::W_MMA;
+                for (int r = 0; ok && item_at(r, it); ++r) {
+                    const int n = it.n;
+                    if (n == 0) continue;
+                    if (!mbar_wait(&bars->kv_full, tn & 1)) break;
+                    tc_fence_after();
+                    const int s0 = gi % C::QS;
+                    if (is_a) {
+                        // A: S^T, dV, dQ.  The item's first S^T overwrites the previous
+                        // item's last once the P/dS warps have read it.
+                        if (gi > 0 && !mbar_wait(&bars->s_free, (gi - 1) & 1)) break;
+                        if (!mbar_wait(&bars->q_full[s0], (gi / C::QS) & 1)) break;
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s0));
+                        mma_commit(&bars->s_full);
+                        for (int i = 0; i < n; ++i) {
+                            const int g = gi + i;  // global iteration: stage and phases
+                            const int s = g % C::QS;
+                            const int s1 = (g + 1) % C::QS;
+                            if (i + 1 < n) {
+                                // S_{i+1} overwrites S_i as soon as the P/dS warps have read it.
+                                if (!mbar_wait(&bars->s_free, g & 1) ||
+                                    !mbar_wait(&bars->q_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
+                                tc_fence_after();
+                                mma_square(tmem + C::COL_S, k_kmaj, q_kmaj + stage_off(s1));
+                                mma_commit(&bars->s_full);
+                            }
+                            if (!mbar_wait(&bars->p_full, g & 1)) { ok = false; break; }
+                            // dV starts from zero in this item: the previous item's epilogue
+                            // must have read it out of TMEM.
+                            if (i == 0 && tn > 0 && !mbar_wait(&bars->dkv_empty, (tn - 1) & 1)) { ok = false; break; }
+                            tc_fence_after();
+                            mma_tmem_a(tmem + C::COL_DV, tmem + C::COL_P, C::P_HALF_STRIDE,
+                                       do_mn + stage_off(s), i > 0);
+                            mma_commit(&bars->p_free);
+                            mma_commit(&bars->stage_empty[s]);  // A's last reader of stage s
+                            // dQ_i over dQ_{i-1}, which the drain has read
+                            if (!mbar_wait(&bars->ds_full, g & 1) ||
+                                (g > 0 && !mbar_wait(&bars->dq_empty, (g - 1) & 1))) { ok = false; break; }
+                            tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_ss(tmem + C::COL_DQ, ds_mn + (uint64_t)(kk * 2048 >> 4),
+                                       k_mn + (uint64_t)(kk * 2048 >> 4), kIdescDq, kk > 0 ? 1u : 0u);
+                            mma_commit(&bars->dq_full);
+                            mma_commit(&bars->ds_empty);
+                        }
+                    } else {
+                        // B: dP^T and dK.  The item's first dP^T follows the previous item's
+                        // last dK in this thread's order (dK read the dS^T it overwrites).
+                        if (!mbar_wait(&bars->do_full[s0], (gi / C::QS) & 1)) break;
+                        tc_fence_after();
+                        mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s0));
+                        mma_commit(&bars->dp_full);
+                        for (int i = 0; i < n; ++i) {
+                            const int g = gi + i;
+                            const int s = g % C::QS;
+                            const int s1 = (g + 1) % C::QS;
+                            if (!mbar_wait(&bars->ds_full, g & 1)) { ok = false; break; }
+                            // dK starts from zero in this item: the previous item's epilogue
+                            // must have read it out of TMEM.
+                            if (i == 0 && tn > 0 && !mbar_wait(&bars->dkv_empty, (tn - 1) & 1)) { ok = false; break; }
+                            tc_fence_after();
+                            mma_tmem_a(tmem + C::COL_DK, tmem + C::COL_DP, C::DS_HALF_STRIDE,
+                                       q_mn + stage_off(s), i > 0);
+                            mma_commit(&bars->stage_empty[s]);  // B's last reader of stage s
+                            if (i + 1 < n) {
+                                // dP^T_{i+1} over dS^T_i, after dK_i in this thread's order
+                                if (!mbar_wait(&bars->do_full[s1], ((g + 1) / C::QS) & 1)) { ok = false; break; }
+                                tc_fence_after();
+                                mma_square(tmem + C::COL_DP, v_kmaj, do_kmaj + stage_off(s1));
+                                mma_commit(&bars->dp_full);
+                            }
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(&bars->dkv_full);
+                    gi += n;
+                    ++tn;
+                }
+            } else {
             for (int r = 0; ok && item_at(r, it); ++r) {
                 const int n = it.n;
                 if (n == 0) continue;
@@ -500,6 +591,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mma_commit(&bars->dkv_full);
                 gi += n;
                 ++tn;
+            }
             }
         }
     } else if (warp >= C::W_DQ0) {
