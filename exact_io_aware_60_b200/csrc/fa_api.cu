@@ -468,8 +468,10 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     const long long grid = std::min<long long>(items, sms);
     // Causal shapes (no key lengths or block mask) with several items per CTA: a balanced
     // static assignment.  Item u is (key tile, head) as the kernel numbers it; its cost is
-    // the query tiles it visits plus about 0.9 of one for its epilogue and the next item's
-    // start (measured on B200).  Without the causal mask every item costs the same.
+    // the query tiles it visits plus the fixed cost of an item (its epilogue and the next
+    // item's start) in units of one query tile: 1.8 at d = 64 (fitted to per-CTA end times
+    // on B200: an item adds 3.1 us, a query tile 1.7 us), 0.9 at d = 128.  Without the
+    // causal mask every item costs the same.
     fa::ItemSchedule sched = no_schedule();
     if (causal && kv_len == nullptr && bmask == nullptr && items > grid &&
         items <= fa::kSchedMaxItems) {
@@ -477,7 +479,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         for (long long u = 0; u < items; ++u) {
             const int kt = (D == 128) ? (int)(u % num_tiles) : (int)(u / bh);
             const int n = causal ? num_tiles - kt : num_tiles;
-            cost[(size_t)u] = (float)n + 0.9f;
+            cost[(size_t)u] = (float)n + (D == 64 ? 1.8f : 0.9f);
         }
         sched = schedule_for({1, D, N, bh, causal ? 1 : 0, grid}, cost, (int)grid);
     }
