@@ -188,7 +188,7 @@ struct BwdCfg {
     static constexpr int OFF_LSE = OFF_DQ + DQ_BYTES;  // QS x 512 B
     static constexpr int OFF_DV = OFF_LSE + QS * 512;  // QS x 512 B
     static constexpr int OFF_BAR = OFF_DV + QS * 512;
-    static constexpr int USED = OFF_BAR + 256;
+    static constexpr int USED = OFF_BAR + 512;  // barriers and the item cache
     // d = 128 uses all 227 KB: no room for alignment slack; the kernel checks instead.
     static constexpr int SLACK = (USED + 1024 <= 232448) ? 1024 : 0;
     static constexpr int SMEM = USED + SLACK;
@@ -224,7 +224,9 @@ struct BwdBars {
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_empty, dq_full, dq_empty,
         dkv_full, dkv_empty;
     uint32_t tmem_base;
+    ItemCache items;  // SCHED: this CTA's list of the launcher's schedule
 };
+static_assert(sizeof(BwdBars) <= 512, "the barrier block has 512 bytes of shared memory");
 
 // DROP: dropout.  With K the keep mask and r = keep_scale, the chain rule gives
 //   dV = r (P o K)^T dO,  dP = r K o (dO V^T),  D = rowsum(dO o O),  dS = P o (dP - D);
@@ -269,6 +271,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // same list on its own.
 
     if (warp == C::W_TMA && lane == 0) {
+        if constexpr (SCHED) item_cache_fill(bars->items, sched);
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -318,9 +321,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     auto item_at = [&](int r, Item &it) -> bool {
         int u;
         if constexpr (SCHED) {  // the launcher's balanced assignment
-            const int b0 = sched.off[blockIdx.x], b1 = sched.off[blockIdx.x + 1];
-            if (r >= b1 - b0) return false;
-            u = sched.ids[b0 + r];
+            if (!item_cache_get(bars->items, sched, r, u)) return false;
         } else {
             const int G = (int)gridDim.x;
             u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
@@ -658,6 +659,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
+        bool store_pending = false;  // the last item's dK/dV stores may still read the dS buffer
         int gi = 0, tn = 0;  // global iteration, items with work so far
         Item it;
         for (int rr = 0; item_at(rr, it); ++rr) {
@@ -776,6 +778,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 break;
             }
             tc_fence_after();
+            if (store_pending) {
+                // the previous item's dK/dV stores have read the dS buffer (this wait
+                // overlapped P_0) before dS_0 goes there
+                if (threadIdx.x == 0) bulk_wait_group_read<0>();
+                named_bar_sync(1, 256);
+                store_pending = false;
+            }
             const float *ndv = sDv + s * 128 + h * 64;  // -D of the 64 queries
             // dS for queries 64h + 32cc .. + 31 from the dP^T values w
             auto ds_half = [&](const uint32_t (&w)[32], int cc) {
@@ -830,6 +839,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                  (!C::DQ_IN_DS || mbar_wait(&bars->dq_stage_free, (gi + n - 1) & 1));
             tc_fence_after();
         }
+        // An item without work has written no dS: the previous stores' reads of the dS
+        // buffer are waited for here, before the staging below (the barrier orders it).
+        if (store_pending && threadIdx.x == 0) bulk_wait_group_read<0>();
+        store_pending = false;
         // Agree again, so that the `break` after the epilogue is taken by all 256 threads
         // or by none (the next item's epilogue barriers need every one of them).
         ok = named_bar_and(1, 256, ok);
@@ -888,14 +901,18 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                      kt * 128, bh);
                 }
                 bulk_commit_group();
-                bulk_wait_group_read<0>();  // the dS buffer is reused right after
+                // The next round reuses the dS buffer right away; after the last round the
+                // next item writes it only for its first dS, which waits then (store_pending).
+                if (round < ROUNDS - 1) bulk_wait_group_read<0>();
             }
-            named_bar_sync(1, 256);
+            if (round < ROUNDS - 1) named_bar_sync(1, 256);
         }
+        store_pending = true;
         gi += n;
         if (n > 0) ++tn;
         if (!ok) break;
         }  // items
+        if (threadIdx.x == 0) bulk_wait_group<0>();  // shared memory must outlive the stores
     }
 
     tc_fence_before();

@@ -108,7 +108,7 @@ struct FwdCfg {
     static constexpr int OFF_K = OFF_Q + QBUF * QTILE;
     static constexpr int OFF_V = OFF_K + NS * KTILE;
     static constexpr int OFF_BAR = OFF_V + NS * VSTAGE;
-    static constexpr int USED = OFF_BAR + 256;
+    static constexpr int USED = OFF_BAR + 512;  // barriers and the item cache
     // Two CTAs per SM leave no room for an alignment pad at d = 64: the kernel checks
     // that the dynamic shared-memory base is 1024-byte aligned instead.
     static constexpr int SLACK = (CTAS_PER_SM == 1) ? 1024 : 0;
@@ -148,7 +148,7 @@ struct FwdCfgF8 {
     static constexpr int OFF_K = OFF_Q + QTILE;
     static constexpr int OFF_V = OFF_K + NS * KTILE;
     static constexpr int OFF_BAR = OFF_V + NS * VSTAGE;
-    static constexpr int USED = OFF_BAR + 256;
+    static constexpr int USED = OFF_BAR + 512;  // barriers and the item cache
     static constexpr int SLACK = 1024;
     static constexpr int SMEM = USED + SLACK;
     static constexpr int THREADS = 192;
@@ -177,6 +177,7 @@ struct FwdBars {
     uint64_t v_full[4];
     uint64_t kv_empty[4];
     uint32_t tmem_base;
+    ItemCache items;  // SCHED: this CTA's list of the launcher's schedule
 };
 
 // DROP: dropout on the probabilities (the mask is regenerated per element from the
@@ -205,12 +206,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
     FwdBars *bars = reinterpret_cast<FwdBars *>(smem + C::OFF_BAR);
-    static_assert(sizeof(FwdBars) <= 256, "barrier area");
+    static_assert(sizeof(FwdBars) <= 512, "barrier area");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 128) {
+        if constexpr (SCHED) item_cache_fill(bars->items, sched);
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -269,9 +271,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     auto item_at = [&](int r, Item &it) -> bool {
         int u;
         if constexpr (SCHED) {  // the launcher's balanced assignment
-            const int b0 = sched.off[blockIdx.x], b1 = sched.off[blockIdx.x + 1];
-            if (r >= b1 - b0) return false;
-            u = sched.ids[b0 + r];
+            if (!item_cache_get(bars->items, sched, r, u)) return false;
         } else {
             const int G = (int)gridDim.x;
             u = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);

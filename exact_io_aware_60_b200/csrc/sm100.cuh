@@ -116,6 +116,29 @@ struct NoSchedule {
     int lists;
 };
 
+// A CTA's own list of a schedule, copied into shared memory once at the start: the
+// schedule is a kernel parameter, and every read of it with a computed index goes to the
+// constant cache and mostly misses (about 1000 cycles for a lookup of the next item,
+// measured on B200).  Lists longer than kItemCache read their remainder from the
+// parameter.
+constexpr int kItemCache = 48;
+struct ItemCache {
+    int b0, n;
+    uint16_t ids[kItemCache];
+};
+__device__ __forceinline__ void item_cache_fill(ItemCache &c, const ItemSchedule &s) {
+    c.b0 = s.off[blockIdx.x];
+    c.n = s.off[blockIdx.x + 1] - c.b0;
+    for (int k = 0; k < c.n && k < kItemCache; ++k) c.ids[k] = s.ids[c.b0 + k];
+}
+// Item r of this CTA's list; false past its end.
+__device__ __forceinline__ bool item_cache_get(const ItemCache &c, const ItemSchedule &s, int r,
+                                               int &u) {
+    if (r >= c.n) return false;
+    u = r < kItemCache ? c.ids[r] : s.ids[c.b0 + r];
+    return true;
+}
+
 // Programmatic dependent launch: kernels of one step are launched so that the next one
 // may start early.  pdl_wait() blocks until the previous kernel in the stream has
 // completed and its memory is visible (it returns at once if there is no such
