@@ -431,7 +431,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         int gj = 0;  // global block count
         Item it;
-        for (int r = 0; item_at(r, it); ++r) {
+        // (the next item is looked up at the start of each item's epilogue and carried over)
+        bool have_item = item_at(0, it);
+        for (int r = 0; have_item; ++r) {
         const int qt = it.qt, bh = it.bh, L = it.L, T = it.T, split = it.split;
         const int row = qt * C::BM + t;
         const bool any_block = it.j_first < T;
@@ -579,7 +581,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
         // ------------------------------ epilogue of the item ---------------------------
         Item nxt;
-        if (!item_at(r + 1, nxt)) pdl_launch_dependents();  // this CTA's last item
+        const bool have_next = item_at(r + 1, nxt);
+        if (!have_next) pdl_launch_dependents();  // this CTA's last item
         if (ok && jj > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, (gj + jj - 1) & 1));
             tc_fence_after();
@@ -642,6 +645,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         if (any_block) gj += jj;
         if (!ok) break;
+        it = nxt;
+        have_item = have_next;
         }  // items
     }
 
