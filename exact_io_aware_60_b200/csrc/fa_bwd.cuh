@@ -29,7 +29,8 @@
 //                    (lane quarter w % 4, query half w / 4): P^T = 2^(S^T scale log2e -
 //                    LSE2), written back to TMEM as 16-bit pairs; dS^T = P^T o (dP^T - D)
 //                    to TMEM and, in the transposed operand layout, to shared memory;
-//                    the item's epilogue writes dK, dV.
+//                    the item's epilogue writes dK, dV (in the non-causal d = 64 variant
+//                    the dQ drain warps write them instead, see BwdCfg::DRAIN_EPI).
 //        warps 10..13 drain dQ_i from TMEM through a swizzled shared-memory staging tile
 //                    and a TMA reduce-add into the fp32 accumulator in global memory (own
 //                    staging area at d = 64; at d = 128, where shared memory is full, the
